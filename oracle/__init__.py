@@ -1,0 +1,9 @@
+"""fp64 CPU oracle for exact attention (test infrastructure, never on the product path).
+
+Only tests, the smoke check and the bench's CPU-baseline leg import this
+package.  It shares no code with the CUDA library.
+"""
+
+from .attention import attention, decode_paged, gather_pages
+
+__all__ = ["attention", "decode_paged", "gather_pages"]

@@ -1,0 +1,154 @@
+"""Plain fp64 CPU oracle for fused exact attention (test infrastructure only).
+
+This module is test infrastructure.  Only ``tests/``, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+it.  The CUDA library never calls it and shares no code with it.
+
+What it computes is the plain definition the fused kernels must reach exactly
+(up to rounding order):
+
+* "FlashAttention (KO)", section "표준 Attention의 문제점" (the problem with
+  standard attention): Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V.  The
+  scale is a caller argument here (1/sqrt(d_k) in that formula; the MLA decode
+  workload passes 1/sqrt(192)).
+* "FlashAttention (KO)", section "온라인 Softmax 계산" (online softmax): the
+  tiled method keeps a running max and a running exp-sum and still reaches the
+  exact softmax result.  So the oracle does NOT tile: it materialises each full
+  row of S = scale * Q K^T and applies the textbook softmax to it.
+* "FlashAttention (KO)", section "단일 CUDA 커널로의 연산 융합" (fusion into one
+  kernel): masking is one of the fused steps.  The only mask here is the causal
+  one, aligned to the bottom-right corner: key j is visible to query i iff
+  j <= i + (Nk - Nq).
+* "GQLA: Group-Query Latent Attention ...", section 1 (MLA) and the
+  "MQA-absorb path" definition: after absorption every query head attends to
+  one shared latent KV row per token.  Here K is the whole 576-wide latent row
+  and V is its first 512 entries.
+* "FlashMLA" page, technical basis list: the KV cache is paged with 64-token
+  pages; a block table maps each sequence's logical page to a physical page.
+
+Outputs: O (fp64) and LSE = ln sum_j exp(S_ij) (fp64, natural log of the sum
+over the *scaled* scores).  A row with no visible key has O = 0, LSE = -inf.
+
+Every value is computed in fp64 from the given input values (the bf16 inputs are
+upcast exactly by the caller).  Row chunking below only bounds memory: each
+chunk holds complete rows of S, so no online rescaling takes place.
+
+Parity pins: tests/test_oracle.py checks this module against hand-derived
+values (tests/golden/), closed forms, invariants, a pure-Python brute force
+and torch's fp64 scaled_dot_product_attention.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["attention", "decode_paged", "gather_pages"]
+
+
+def _rows_softmax_weighted(S: np.ndarray, V: np.ndarray):
+    """Textbook softmax of each row of S applied to V.
+
+    Returns (O, LSE).  S holds -inf for masked entries.  Rows whose entries are
+    all -inf give O = 0 and LSE = -inf (no visible key).
+    """
+    m = np.max(S, axis=1, keepdims=True)
+    empty = ~np.isfinite(m[:, 0])
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    P = np.exp(S - m_safe)                      # exp(-inf) = 0 for masked keys
+    l = np.sum(P, axis=1, keepdims=True)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        O = (P @ V) / l
+        lse = m_safe[:, 0] + np.log(l[:, 0])
+    O[empty] = 0.0
+    lse[empty] = -np.inf
+    return O, lse
+
+
+def attention(q, k, v, causal: bool, scale: float, q_rows=None, row_chunk: int = 1024):
+    """Exact attention, one (batch, query head) at a time, S materialised.
+
+    q: [B, Nq, Hq, D]; k: [B, Nk, Hkv, D]; v: [B, Nk, Hkv, Dv] (any real dtype,
+    upcast to fp64).  Query head hq reads KV head hq // (Hq // Hkv) (contiguous
+    groups; grouped-query attention with Hkv = 1 is multi-query attention).
+
+    q_rows: optional 1-D array of query row indices; only those rows are
+    computed (for spot checks at full size).  Returns O [B, len(rows), Hq, Dv]
+    and LSE [B, Hq, len(rows)] in fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, Dk = k.shape
+    Dv = v.shape[3]
+    assert Dk == D and v.shape[:3] == (B, Nk, Hkv)
+    assert Hq % Hkv == 0
+    group = Hq // Hkv
+    rows = np.arange(Nq) if q_rows is None else np.asarray(q_rows, dtype=np.int64)
+    R = rows.shape[0]
+    O = np.zeros((B, R, Hq, Dv), dtype=np.float64)
+    LSE = np.full((B, Hq, R), -np.inf, dtype=np.float64)
+    if Nk == 0 or R == 0:
+        return O, LSE
+    key_idx = np.arange(Nk)
+    for b in range(B):
+        for hq in range(Hq):
+            kv = hq // group
+            Kmat = k[b, :, kv, :]
+            Vmat = v[b, :, kv, :]
+            for c0 in range(0, R, row_chunk):
+                r = rows[c0:c0 + row_chunk]
+                S = scale * (q[b, r, hq, :] @ Kmat.T)
+                if causal:
+                    visible = key_idx[None, :] <= (r[:, None] + (Nk - Nq))
+                    S = np.where(visible, S, -np.inf)
+                o, lse = _rows_softmax_weighted(S, Vmat)
+                O[b, c0:c0 + len(r), hq, :] = o
+                LSE[b, hq, c0:c0 + len(r)] = lse
+    return O, LSE
+
+
+def gather_pages(kv_pages, block_table_row, seqlen: int, page_size: int):
+    """Tokens 0..seqlen-1 of one sequence, read through its block-table row.
+
+    kv_pages: [num_pages, page_size, Dk].  Token t lives in physical page
+    block_table_row[t // page_size], row t % page_size.
+    """
+    kv_pages = np.asarray(kv_pages)
+    out = np.empty((seqlen, kv_pages.shape[-1]), dtype=np.float64)
+    for t0 in range(0, seqlen, page_size):
+        page = int(block_table_row[t0 // page_size])
+        n = min(page_size, seqlen - t0)
+        out[t0:t0 + n] = kv_pages[page, :n, :]
+    return out
+
+
+def decode_paged(q, kv_pages, block_table, cache_seqlens, scale: float, dv: int,
+                 page_size: int = 64, heads=None):
+    """MLA absorbed decode over a paged latent cache (one query token per sequence).
+
+    q: [B, Hq, Dk] absorbed queries; kv_pages: [num_pages, page_size, Dk] latent
+    rows; block_table: [B, max_pages] int; cache_seqlens: [B] int.
+    K = the gathered latent rows (all Dk entries), V = their first ``dv``
+    entries; every query head attends to the same K/V (MQA-absorb form), no
+    mask within the sequence (the single new token sees all cached tokens).
+    heads: optional subset of query heads.  Returns O [B, len(heads), dv] and
+    LSE [B, len(heads)] in fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kv_pages = np.asarray(kv_pages, dtype=np.float64)
+    B, Hq, Dk = q.shape
+    hs = np.arange(Hq) if heads is None else np.asarray(heads, dtype=np.int64)
+    O = np.zeros((B, len(hs), dv), dtype=np.float64)
+    LSE = np.full((B, len(hs)), -np.inf, dtype=np.float64)
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        if L == 0:
+            continue
+        Kmat = gather_pages(kv_pages, block_table[b], L, page_size)
+        Vmat = Kmat[:, :dv]
+        S = scale * (q[b, hs, :] @ Kmat.T)
+        o, lse = _rows_softmax_weighted(S, Vmat)
+        O[b] = o
+        LSE[b] = lse
+    return O, LSE
