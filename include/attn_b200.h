@@ -1,0 +1,137 @@
+/*
+ * attn_b200.h: C ABI of the B200 (sm_100a) fused exact-attention library.
+ *
+ * Two operations, both computing  O = softmax(scale * Q K^T + mask) V  and the
+ * per-row log-sum-exp, exactly (up to floating-point rounding), without ever
+ * writing the score matrix to device memory:
+ *
+ *   attn_fwd           prefill / training forward over dense Q, K, V
+ *   attn_decode_paged  one-token MLA ("MQA-absorb") decode over a paged cache
+ *
+ * Sources for what is computed (web pages, cited by title and section):
+ *   - "FlashAttention (KO)", section on the problems of standard attention:
+ *     Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V; the N x N matrix S is
+ *     what the IO-aware method never stores.
+ *   - same page, sections on tiling, online softmax (running max and running
+ *     exp-sum reach the exact result) and fusion of QK^T, masking, softmax
+ *     and the product with V into one kernel.
+ *   - "FlashMLA" page, technical basis: BF16, variable-length sequences, a KV
+ *     cache paged in 64-token pages.
+ *   - "GQLA: Group-Query Latent Attention ...", sections 1-3: MLA compresses K
+ *     and V into one low-rank latent; in the MQA-absorb decode path every
+ *     query head attends to that one shared latent.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are device pointers, contiguous, row-major, bf16 unless
+ *     stated; the caller owns every buffer (allocates and frees it).  The
+ *     library allocates no device memory except one status word per device,
+ *     created on first use.
+ *   - Calls only enqueue work on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and return; they never synchronise.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and leave every output untouched.
+ *   - Nothing is thrown across the ABI; every call returns an attn_status.
+ *   - A kernel that finds a barrier phase stuck for more than 2 s aborts,
+ *     frees its tensor memory, and records ATTN_ERR_TIMEOUT in the device
+ *     status word (read it with attn_read_device_status after synchronising).
+ */
+#ifndef ATTN_B200_H_
+#define ATTN_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or scale    */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what is implemented     */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed   */
+  ATTN_ERR_TIMEOUT = 4,     /* device-side bounded wait expired (status word)*/
+  ATTN_ERR_WORKSPACE = 5    /* workspace missing or smaller than required    */
+} attn_status;
+
+/* Version of this ABI; bumped on any incompatible change. */
+int attn_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_fwd: fused exact attention forward.
+ *
+ *   q   [B, Nq, Hq,  D ] bf16      k [B, Nk, Hkv, D] bf16
+ *   v   [B, Nk, Hkv, Dv] bf16      o [B, Nq, Hq, Dv] bf16 (written)
+ *   lse [B, Hq, Nq]      fp32 (written): natural log of sum_j exp(scale*q_i.k_j)
+ *       over the visible keys j.
+ *
+ * Query head h reads KV head h / (Hq / Hkv) (grouped-query attention; Hkv = 1
+ * is multi-query attention, Hkv = Hq multi-head).
+ * causal != 0 masks key j for query i when j > i + (Nk - Nq) (mask aligned to
+ * the bottom-right corner; the usual lower triangle when Nq == Nk).  A query
+ * row with no visible key gets O = 0 and LSE = -inf.
+ *
+ * Supported: D == Dv in {64, 128, 256}; Hq % Hkv == 0; scale finite and > 0;
+ * q, k, v, o 16-byte aligned; lse 4-byte aligned; Nq, Nk >= 0, B, Hq, Hkv >= 1,
+ * B and Hq at most 65535.  Accumulation is fp32; probabilities are rounded to
+ * bf16 before the product with V; O is rounded to bf16 once at the end.
+ * Results are deterministic run to run.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+             int Nk, int D, int Dv, int causal, float scale, void* stream);
+
+/*
+ * attn_decode_paged_workspace_size: bytes of device workspace that
+ * attn_decode_paged needs for a batch of B sequences with Hq heads of width
+ * Dv on the current device.  The caller allocates it (any alignment >= 256 B).
+ */
+size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv);
+
+/*
+ * attn_decode_paged: one new query token per sequence attending to a paged
+ * latent KV cache, MLA absorbed ("MQA-absorb") form.
+ *
+ *   q             [B, 1, Hq, Dk] bf16   absorbed queries
+ *   kv_pages      [num_pages, page_size, 1, Dk] bf16 latent rows; K = all Dk
+ *                 entries of a row, V = its first Dv entries
+ *   block_table   [B, max_pages_per_seq] int32: token t of sequence b lives in
+ *                 page block_table[b][t / page_size], row t % page_size
+ *   cache_seqlens [B] int32: number of cached tokens of each sequence
+ *   o             [B, 1, Hq, Dv] bf16 (written)
+ *   lse           [B, Hq] fp32 (written), natural-log LSE of the scaled scores
+ *   workspace     device scratch of at least attn_decode_paged_workspace_size
+ *                 bytes (split-KV partial results); its content on entry is
+ *                 irrelevant and undefined on return.
+ *
+ * The new token sees every cached token of its sequence (no mask inside the
+ * length).  A sequence of length 0 gets O = 0 and LSE = -inf.  Rows of a page
+ * past the sequence length and pages past its last page are never used in
+ * the result, but must hold finite values (they may be read).
+ *
+ * Supported: Dk = 576, Dv = 512, page_size = 64, Hq = 128; block-table
+ * entries in [0, num_pages) for every page a sequence uses; lengths in
+ * [0, max_pages_per_seq * page_size]; pointers 16-byte aligned.
+ * Lengths and block-table entries are read on the device (no host sync); out
+ * of range entries make the kernel skip that sequence and record
+ * ATTN_ERR_INVALID_ARG in the device status word.
+ */
+int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_table,
+                      const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk, int Dv,
+                      int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * attn_read_device_status: status recorded by kernels on `device` since the
+ * last call (ATTN_OK if none), then reset to ATTN_OK.  Synchronises with the
+ * device first.  Returns ATTN_ERR_CUDA if the device cannot be queried.
+ */
+int attn_read_device_status(int device);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H_ */

@@ -1,0 +1,57 @@
+"""Shared comparison helpers for the GPU parity tests.
+
+Tolerances (bf16 inputs, fp32 accumulation), against the unrounded fp64 oracle:
+  O:   max |O - O*| <= 1e-2  and  ||O - O*||_2 / ||O*||_2 <= 5e-3
+  LSE: max |LSE - LSE*| <= 1e-3 over rows with a visible key; rows with none
+       must be -inf on both sides.
+"""
+
+import json
+import os
+
+import numpy as np
+import torch
+
+O_MAX_ABS = 1e-2
+O_REL_RMS = 5e-3
+LSE_MAX_ABS = 1e-3
+
+
+def to_np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def bf16_arith_bound(v_absmax: float) -> float:
+    """Worst-case O error of the kernel's own bf16 roundings, for inputs far
+    from the workloads' N(0,1) rows (peaked softmax, large |V|).
+
+    Each probability is rounded to bf16 (relative error <= 2^-8) before the
+    product with V, so O moves by at most 2^-8 * max|V|; the final rounding of
+    O to bf16 adds at most 2^-8 * |O| <= 2^-8 * max|V|.  Total 2^-7 * max|V|.
+    """
+    return 2.0 ** -7 * v_absmax
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, what="", o_max_abs=O_MAX_ABS):
+    o = to_np64(o_gpu) if isinstance(o_gpu, torch.Tensor) else np.asarray(o_gpu, np.float64)
+    lse = to_np64(lse_gpu) if isinstance(lse_gpu, torch.Tensor) else np.asarray(lse_gpu, np.float64)
+    assert o.shape == o_ref.shape, (o.shape, o_ref.shape)
+    assert lse.shape == lse_ref.shape, (lse.shape, lse_ref.shape)
+    assert np.all(np.isfinite(o)), f"{what}: non-finite O"
+    err = np.abs(o - o_ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    ref_norm = float(np.linalg.norm(o_ref))
+    rel_rms = float(np.linalg.norm(o - o_ref) / ref_norm) if ref_norm > 0 else float(np.linalg.norm(o))
+    ref_empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), ref_empty), f"{what}: -inf LSE rows differ"
+    fin = ~ref_empty
+    lse_err = float(np.abs(lse[fin] - lse_ref[fin]).max()) if fin.any() else 0.0
+    stats = dict(max_abs=max_abs, rel_rms=rel_rms, lse_max_abs=lse_err)
+    log = os.environ.get("PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps(dict(case=what, **stats)) + "\n")
+    assert max_abs <= o_max_abs, f"{what}: O max-abs {max_abs:.3e} > {o_max_abs} {stats}"
+    assert rel_rms <= O_REL_RMS, f"{what}: O rel-RMS {rel_rms:.3e} > {O_REL_RMS} {stats}"
+    assert lse_err <= LSE_MAX_ABS, f"{what}: LSE max-abs {lse_err:.3e} > {LSE_MAX_ABS} {stats}"
+    return stats

@@ -1,0 +1,69 @@
+"""C-ABI checks that need no GPU: the library loads, exports what the header
+declares, and rejects bad arguments on the host before touching CUDA."""
+
+import ctypes
+
+import pytest
+
+import exact_attention_135_b200 as ea
+from exact_attention_135_b200 import build as ea_build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ea_build.build()
+    return ea.library()
+
+
+def test_header_symbols_exported(lib):
+    names = ea.exported_symbols()
+    assert {"attn_fwd", "attn_decode_paged", "attn_decode_paged_workspace_size", "attn_status_string",
+            "attn_read_device_status", "attn_abi_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+
+
+def test_status_strings(lib):
+    assert lib.attn_abi_version() == 1
+    for code, name in ea.STATUS.items():
+        assert lib.attn_status_string(code).decode() == name
+    assert lib.attn_status_string(99).decode() == "ATTN_ERR_UNKNOWN"
+
+
+A = 0x10000   # fake 16-byte aligned addresses: never dereferenced on the error paths below
+
+
+def _fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=2, Nq=128, Nk=128, D=64, Dv=64, causal=0, scale=0.125):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, Dv, causal, scale, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert _fwd(lib, q=None) == 1
+    assert _fwd(lib, lse=None) == 1
+    assert _fwd(lib, k=A + 8) == 1            # misaligned
+    assert _fwd(lib, lse=A + 2) == 1
+    assert _fwd(lib, Hq=3, Hkv=2) == 1        # Hq % Hkv
+    assert _fwd(lib, B=0) == 1
+    assert _fwd(lib, Nq=-1) == 1
+    assert _fwd(lib, scale=0.0) == 1
+    assert _fwd(lib, scale=-1.0) == 1
+    assert _fwd(lib, scale=float("nan")) == 1
+    assert _fwd(lib, scale=float("inf")) == 1
+    assert _fwd(lib, B=70000) == 1
+
+
+def test_fwd_unsupported_shapes(lib):
+    assert _fwd(lib, D=96, Dv=96) == 2
+    assert _fwd(lib, D=128, Dv=64) == 2
+    assert _fwd(lib, D=32, Dv=32) == 2
+
+
+def test_fwd_empty_query_is_noop(lib):
+    assert _fwd(lib, Nq=0) == 0
+
+
+def test_fwd_no_keys_accepts_null_kv_and_empty_query(lib):
+    # Nq == 0: nothing to do, no CUDA call, even with null K/V
+    assert _fwd(lib, k=None, v=None, Nq=0, Nk=0) == 0
+    # Nk > 0 with null K is an argument error
+    assert _fwd(lib, k=None, Nk=5) == 1
