@@ -106,7 +106,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def prefill_setup(dev):
+class Part:
+    """One timed piece of the step: a callable on device-resident inputs plus
+    its end-to-end variant (pinned host inputs copied in, result copied out)."""
+
+    def __init__(self, name, run, h2d, d2h, launches):
+        self.name, self.run, self.h2d, self.d2h, self.launches = name, run, h2d, d2h, launches
+
+    def e2e(self):
+        for dst, src in self.h2d:
+            dst.copy_(src, non_blocking=True)
+        self.run()
+        for dst, src in self.d2h:
+            dst.copy_(src, non_blocking=True)
+
+    def bytes(self, pairs):
+        return sum(a.numel() * a.element_size() for a, _ in pairs)
+
+
+def prefill_part(ea, dev):
     cfg = inputs.PREFILL_CONFIGS[PREFILL_ID]
     q, k, v = inputs.prefill_config_inputs(cfg)
     host = {"q": q.pin_memory(), "k": k.pin_memory(), "v": v.pin_memory()}
@@ -115,7 +133,78 @@ def prefill_setup(dev):
     d["lse"] = torch.empty((cfg.B, cfg.Hq, cfg.Nq), dtype=torch.float32, device=dev)
     host["o"] = torch.empty(d["o"].shape, dtype=torch.bfloat16).pin_memory()
     host["lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
-    return cfg, host, d
+
+    def run():
+        ea.fwd(d["q"], d["k"], d["v"], causal=cfg.causal, scale=cfg.scale, out=d["o"], lse=d["lse"])
+
+    p = Part("prefill", run, [(d[n], host[n]) for n in ("q", "k", "v")],
+             [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=1)
+    p.cfg = cfg
+    p.work = cfg.flops()
+    return p
+
+
+def decode_part(ea, dev):
+    cfg = inputs.DECODE_CONFIG
+    c = inputs.decode_config_inputs(cfg)
+    host = {"q": c.q.pin_memory(), "kv": c.kv_pages.pin_memory(), "bt": c.block_table.pin_memory(),
+            "sl": c.cache_seqlens.pin_memory()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    d["o"] = torch.empty((cfg.B, 1, cfg.Hq, cfg.Dv), dtype=torch.bfloat16, device=dev)
+    d["lse"] = torch.empty((cfg.B, cfg.Hq), dtype=torch.float32, device=dev)
+    d["ws"] = torch.empty(ea.decode_workspace_size(cfg.B, cfg.Hq, cfg.Dv, dev), dtype=torch.uint8, device=dev)
+    host["o"] = torch.empty(d["o"].shape, dtype=torch.bfloat16).pin_memory()
+    host["lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
+
+    def run():
+        ea.decode_paged(d["q"], d["kv"], d["bt"], d["sl"], cfg.scale, dv=cfg.Dv, out=d["o"], lse=d["lse"],
+                        workspace=d["ws"])
+
+    p = Part("decode", run, [(d[n], host[n]) for n in ("q", "kv", "bt", "sl")],
+             [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=2)
+    p.cfg = cfg
+    p.kv_bytes = c.kv_valid_bytes(cfg.Dk)
+    p.tokens = int(c.cache_seqlens.to(torch.int64).sum())
+    p.flops = 2.0 * cfg.Hq * (cfg.Dk + cfg.Dv) * p.tokens
+    p.ws_bytes = d["ws"].numel()
+    return p
+
+
+def time_parts(parts, steps, stream):
+    """Times `steps` steps; each step runs every part once.  Returns total ms
+    and per-part lists of per-launch ms (CUDA events on the launching stream)."""
+    ev = {p.name: [] for p in parts}
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    pairs = {p.name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(steps)] for p in parts}
+    t0.record(stream)
+    for i in range(steps):
+        for p in parts:
+            a, b = pairs[p.name][i]
+            a.record(stream)
+            p.run()
+            b.record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    for p in parts:
+        ev[p.name] = [a.elapsed_time(b) for a, b in pairs[p.name]]
+    return t0.elapsed_time(t1), ev
+
+
+def time_e2e(parts, steps, warmup, dev, stream):
+    out = {p.name: [] for p in parts}
+    for p in parts:
+        for i in range(warmup + steps):
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            p.e2e()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= warmup:
+                out[p.name].append(a.elapsed_time(b))
+    return out
 
 
 def run_gpu(args):
@@ -130,15 +219,17 @@ def run_gpu(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     peaks, peaks_kind = load_peaks()
-
-    cfg, host, d = prefill_setup(dev)
     stream = torch.cuda.current_stream(dev)
 
-    def prefill():
-        ea.fwd(d["q"], d["k"], d["v"], causal=cfg.causal, scale=cfg.scale, out=d["o"], lse=d["lse"])
+    parts = []
+    if args.part in ("all", "prefill"):
+        parts.append(prefill_part(ea, dev))
+    if args.part in ("all", "decode"):
+        parts.append(decode_part(ea, dev))
 
     for _ in range(args.warmup):
-        prefill()
+        for p in parts:
+            p.run()
     torch.cuda.synchronize(dev)
     if ea.read_device_status(dev.index) != 0:
         raise RuntimeError("device status error after warm-up")
@@ -149,81 +240,80 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t_all0 = torch.cuda.Event(enable_timing=True)
-    t_all1 = torch.cuda.Event(enable_timing=True)
-    t_all0.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        prefill()
-        ev[i][1].record(stream)
-    t_all1.record(stream)
-    torch.cuda.synchronize(dev)
+    total_ms, per = time_parts(parts, args.steps, stream)
     clocks = sampler.stop()
     if world > 1:
         torch.distributed.barrier()
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = t_all0.elapsed_time(t_all1)
     if ea.read_device_status(dev.index) != 0:
         raise RuntimeError("device status error in timed region")
+    e2e = time_e2e(parts, args.e2e_steps, 3, dev, stream)
 
-    # end to end through the public API, host buffers, copies inside the timed region
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for n in ("q", "k", "v"):
-            d[n].copy_(host[n], non_blocking=True)
-        prefill()
-        host["o"].copy_(d["o"], non_blocking=True)
-        host["lse"].copy_(d["lse"], non_blocking=True)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
-    d2h = sum(host[n].numel() * host[n].element_size() for n in ("o", "lse"))
-
-    flops = cfg.flops()
-    step_ms = total_ms / args.steps
-    e2e_step = sum(e2e_ms) / len(e2e_ms)
+    # max over ranks of every timing
+    names = [p.name for p in parts]
+    vec = [total_ms / args.steps] + [statistics.mean(per[n]) for n in names] + \
+          [statistics.mean(e2e[n]) for n in names]
     if world > 1:
-        t = torch.tensor([step_ms, e2e_step, statistics.mean(launch_ms)], device=dev)
+        t = torch.tensor(vec, device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, e2e_step, avg_launch = t.tolist()
+        vec = t.tolist()
+    step_ms = vec[0]
+    launch_ms = dict(zip(names, vec[1:1 + len(names)]))
+    e2e_ms = dict(zip(names, vec[1 + len(names):]))
+    by = {p.name: p for p in parts}
+
+    line = {"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: i.i.d. N(0,1) bf16 from a seeded CPU generator",
+            "gpu_launches": args.steps * sum(p.launches for p in parts), "clocks": clocks}
+    step_parts = "+".join(names)
+    decode_obj = None
+    if "decode" in by:
+        p = by["decode"]
+        gbs = p.kv_bytes / (launch_ms["decode"] * 1e-3) / 1e9
+        decode_obj = {
+            "metric": "KV-cache GB/s (paged decode)", "value": round(world * gbs, 1), "unit": "GB/s",
+            "ms_per_launch": round(launch_ms["decode"], 4),
+            "config": {"workload": p.cfg.name, "B": p.cfg.B, "Hq": p.cfg.Hq, "Dk": p.cfg.Dk, "Dv": p.cfg.Dv,
+                       "page_size": p.cfg.page_size, "lengths": f"uniform [{p.cfg.min_len}, {p.cfg.max_len}]",
+                       "tokens": p.tokens, "kv_bytes": p.kv_bytes, "scale": p.cfg.scale,
+                       "l2": "KV cache 340 MB per step, larger than L2, no flush"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
+                         "traffic": None, "kernel": "decode_split_kernel + decode_combine_kernel",
+                         "tflops": round(p.flops / (launch_ms["decode"] * 1e-3) / 1e12, 1),
+                         "tensor_frac": round(p.flops / (launch_ms["decode"] * 1e-3) / 1e12 /
+                                              peaks["bf16_tflops"], 4)},
+            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["decode"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+            "workspace_bytes": p.ws_bytes,
+        }
+    if "prefill" in by:
+        p = by["prefill"]
+        achieved = p.work / (launch_ms["prefill"] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        line.update({
+            "metric": "attention TFLOP/s (prefill)",
+            "value": round(world * p.work / (launch_ms["prefill"] * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "config": {"workload": p.cfg.name, "step": step_parts, "B": p.cfg.B, "Hq": p.cfg.Hq,
+                       "Hkv": p.cfg.Hkv, "Nq": p.cfg.Nq, "Nk": p.cfg.Nk, "D": p.cfg.D, "causal": p.cfg.causal,
+                       "scale": p.cfg.scale, "global_batch": p.cfg.B * world, "seq_len": p.cfg.Nq,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (Q 134 MB + K/V 67 MB per step), no flush"},
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": f"{peaks_kind} bf16 burst",
+                         "traffic": None, "kernel": "attn_fwd_kernel<D=128,causal>",
+                         "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)},
+            "e2e": {"value": round(world * p.work / (e2e_ms["prefill"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+        })
+        if decode_obj:
+            line["decode"] = decode_obj
     else:
-        avg_launch = statistics.mean(launch_ms)
-    value = world * flops / (step_ms * 1e-3) / 1e12
-    achieved = flops / (avg_launch * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
-    line = {
-        "metric": "attention TFLOP/s (prefill)",
-        "value": round(value, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(step_ms, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic: i.i.d. N(0,1) bf16 from a seeded CPU generator",
-        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Nq": cfg.Nq, "Nk": cfg.Nk,
-                   "D": cfg.D, "causal": cfg.causal, "scale": cfg.scale, "global_batch": cfg.B * world,
-                   "seq_len": cfg.Nq, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q 134 MB + K/V 67 MB per step), no flush"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": f"{peaks_kind} bf16 burst",
-                     "traffic": None, "kernel": "attn_fwd_kernel<D=128,causal>"},
-        "e2e": {"value": round(world * flops / (e2e_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
-        "clocks": clocks,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+        line.update({k: decode_obj[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
+        line["config"]["step"] = step_parts
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and "prefill" in by:
+        line["cpu_baseline"] = cpu_baseline(args.baseline_rows)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -231,21 +321,28 @@ def run_gpu(args):
         print(json.dumps(line), flush=True)
 
 
+_ORACLE_INPUTS = {}
+
+
 def oracle_prefill_sample(cfg, rows_per_head: int, seed: int):
-    """Time the fp64 oracle on `rows_per_head` random query rows of every head."""
+    """Time the fp64 oracle on `rows_per_head` random query rows of every head.
+
+    Returns (algorithmic FLOPs of the sampled rows, seconds, rows).  The inputs
+    are drawn and upcast once per process, outside the timed region.
+    """
     import numpy as np
     import oracle
 
-    q, k, v = inputs.prefill_config_inputs(cfg)
-    q64 = q.to(torch.float64).numpy()
-    k64 = k.to(torch.float64).numpy()
-    v64 = v.to(torch.float64).numpy()
+    if cfg.name not in _ORACLE_INPUTS:
+        q, k, v = inputs.prefill_config_inputs(cfg)
+        _ORACLE_INPUTS[cfg.name] = tuple(t.to(torch.float64).numpy() for t in (q, k, v))
+    q64, k64, v64 = _ORACLE_INPUTS[cfg.name]
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(cfg.Nq, size=rows_per_head, replace=False))
     t0 = time.perf_counter()
     oracle.attention(q64, k64, v64, cfg.causal, cfg.scale, q_rows=rows)
     dt = time.perf_counter() - t0
-    # algorithmic FLOPs of the sampled rows under the workload's own count
+    # the sampled rows' share of the workload's FLOP count (4*Nq*Nk*D per head, halved when causal)
     share = rows_per_head / cfg.Nq
     return cfg.flops() * share, dt, rows
 
@@ -305,11 +402,17 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=8, help="query rows per head in each oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=64,
+                    help="query rows per head in each step of --impl reference")
+    ap.add_argument("--baseline-rows", type=int, default=768,
+                    help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all",
+                    help="time only one piece of the step (for profiling runs)")
+    ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -1,16 +1,626 @@
-// Paged MLA decode (MQA-absorb form): split-KV kernel plus LSE combine.
+// Paged MLA decode, "MQA-absorb" form, for sm_100a (B200).
+//
+// What it computes: for each sequence b, one absorbed query token with Hq=128
+// heads attends to the L_b cached latent rows of that sequence (pages of 64
+// tokens reached through the block table; "FlashMLA" page: BF16, paged KV
+// with 64-token pages, variable lengths).  Every head reads the same latent
+// row ("GQLA" page, MQA-absorb path): K = the whole 576-wide row, V = its
+// first 512 entries.  O = softmax(scale * q K^T) V and LSE per (b, head).
+//
+// Work split (split-KV): the pages of all sequences are laid end to end and
+// cut into one contiguous, page-aligned range per CTA pair, so every pair
+// reads the same number of pages whatever the length mix.  A range covers
+// the tail of one sequence, whole sequences, and the head of another.  A
+// sequence read entirely by one pair is written out directly; the pieces of
+// a sequence shared by several pairs are written as fp32 partial results
+// (O normalised by its own sum, plus its LSE) and merged by the LSE-combine
+// kernel:  lse = ln sum_i exp(lse_i),  O = sum_i exp(lse_i - lse) O_i
+// (the identity behind the running max / running sum of the online softmax,
+// "FlashAttention (KO)", online softmax section).
+//
+// The accumulator of 128 heads x 512 fp32 fills all 512 TMEM columns of an
+// SM, so the two CTAs of a pair split the 512 output columns: CTA r owns
+// columns [256 r, 256 r + 256).  Each CTA computes the full 128 x 64 score
+// tile per page itself.  TMEM columns per CTA:
+//   [0,256) O half | [256,320) S | [320,352) P (bf16) | [352,512) Q dims 256..575
+// Q dims 0..255 sit in shared memory (64 KB) next to a 2-stage ring of whole
+// pages (2 x 72 KB).
+#include <math.h>
+
 #include "host_common.h"
+#include "sm100.cuh"
+
+namespace ea {
+
+namespace dec {
+
+constexpr int HQ = 128;
+constexpr int DK = 576;
+constexpr int DV = 512;
+constexpr int PAGE = 64;
+constexpr int B_MAX = 2048;
+constexpr int STAGES = 2;
+constexpr int CHUNKS = DK / 64;                 // 9 column chunks of 128 bytes
+constexpr int Q_SMEM_CHUNKS = 4;                // dims 0..255 in shared memory
+constexpr int Q_TMEM_DIMS = DK - 64 * Q_SMEM_CHUNKS;   // 320 dims in TMEM
+constexpr int Q_CHUNK_BYTES = HQ * 128;         // 16 KB
+constexpr int PAGE_CHUNK_BYTES = PAGE * 128;    // 8 KB
+constexpr int Q_BYTES = Q_SMEM_CHUNKS * Q_CHUNK_BYTES;
+constexpr int STAGE_BYTES = CHUNKS * PAGE_CHUNK_BYTES;  // 72 KB
+constexpr int O_COL = 0;
+constexpr int S_COL = 256;
+constexpr int P_COL = 320;
+constexpr int Q_COL = 352;
+constexpr int TMEM_COLS = 512;
+constexpr int THREADS = 192;                    // 4 softmax warps, producer, MMA
+constexpr int PRODUCER_WARP = 4;
+constexpr int MMA_WARP = 5;
+// barriers
+constexpr int B_QF = 0, B_QE = 1, B_QT = 2, B_KF = 3, B_KE = B_KF + STAGES, B_SF = B_KE + STAGES;
+constexpr int B_SE = B_SF + 1, B_PF = B_SE + 1, B_OD = B_PF + 1, B_OF = B_OD + 1, B_DR = B_OF + 1;
+constexpr int NBAR = B_DR + 1;
+// shared memory
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + Q_BYTES;
+constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int OFF_PREF = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_PREF + (B_MAX + 1) * 4 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct Args {
+  const __nv_bfloat16* q;        // [B, Hq, DK]
+  const int32_t* block_table;    // [B, max_pages]
+  const int32_t* seqlens;        // [B]
+  __nv_bfloat16* o;              // [B, Hq, DV]
+  float* lse;                    // [B, Hq]
+  int32_t* ws_pref;              // [B + 1]
+  float* ws_lse;                 // [2 * pairs, Hq]
+  float* ws_o;                   // [2 * pairs, Hq, DV]
+  int* status;
+  int B, max_pages, num_pages, pairs;
+  float scale_log2;
+};
+
+// Pages a sequence contributes (its length clamped to the block table).
+__device__ __forceinline__ int seq_pages(int L, int max_pages) {
+  if (L <= 0) return 0;
+  const int n = (L + PAGE - 1) / PAGE;
+  return n < max_pages ? n : max_pages;
+}
+
+__device__ __forceinline__ int seq_len_eff(int L, int max_pages) {
+  if (L <= 0) return 0;
+  const int cap = max_pages * PAGE;
+  return L < cap ? L : cap;
+}
+
+// First page of pair p's range: floor(p * T / pairs).
+__device__ __forceinline__ int range_start(int p, int T, int pairs) {
+  return (int)(((long long)p * T) / pairs);
+}
+
+// Pair whose range holds global page g (0 <= g < T).
+__device__ __forceinline__ int pair_of_page(int g, int T, int pairs) {
+  return (int)((((long long)g + 1) * pairs - 1) / T);
+}
+
+// Walks the segments (b, first global page, end global page) of [R0, R1).
+struct SegWalk {
+  const int* pref;
+  int B, R0, R1, b;
+  __device__ void init(const int* pref_, int B_, int R0_, int R1_) {
+    pref = pref_;
+    B = B_;
+    R0 = R0_;
+    R1 = R1_;
+    // last b with pref[b] <= R0 (binary search over the prefix sums)
+    int lo = 0, hi = B;   // invariant: pref[lo] <= R0, answer in [lo, hi)
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pref[mid] <= R0) lo = mid; else hi = mid;
+    }
+    b = lo;
+  }
+  // Next non-empty segment; false when the range is exhausted.
+  __device__ bool next(int& sb, int& g0, int& g1) {
+    while (b < B && pref[b] < R1) {
+      const int s = max(R0, pref[b]), e = min(R1, pref[b + 1]);
+      const int cur = b++;
+      if (e > s) {
+        sb = cur;
+        g0 = s;
+        g1 = e;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                        const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + OFF_MISC + 4);
+  int* pref = reinterpret_cast<int*>(base_ptr + OFF_PREF);
+  auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8u * i; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x >> 1;
+  const int half = blockIdx.x & 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QF), 1);
+    mbar_init(bar(B_QE), 1);
+    mbar_init(bar(B_QT), 4);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar(B_KF + s), 1);
+      mbar_init(bar(B_KE + s), 1);
+    }
+    mbar_init(bar(B_SF), 1);
+    mbar_init(bar(B_SE), 4);
+    mbar_init(bar(B_PF), 4);
+    mbar_init(bar(B_OD), 1);
+    mbar_init(bar(B_OF), 4);
+    mbar_init(bar(B_DR), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  // prefix sums of pages per sequence (one pass by warp 0; B <= B_MAX)
+  if (warp == 0) {
+    int carry = 0;
+    bool bad = false;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      int n = 0;
+      if (b < a.B) {
+        const int L = a.seqlens[b];
+        n = seq_pages(L, a.max_pages);
+        bad |= (L < 0) || ((long long)L > (long long)a.max_pages * PAGE);
+      }
+      int x = n;   // inclusive warp scan
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (b < a.B) pref[b + 1] = carry + x;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) pref[0] = 0;
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
+  }
+  if (warp == PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int T = pref[a.B];
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= a.B; i += THREADS) a.ws_pref[i] = pref[i];
+  const int R0 = range_start(pair, T, a.pairs), R1 = range_start(pair + 1, T, a.pairs);
+
+  if (warp == PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      SegWalk w;
+      w.init(pref, a.B, R0, R1);
+      int sb, g0, g1, seg = 0, g = 0;
+      bool ok = true;
+      int issued = 0;
+      int q_last = -1;
+      while (ok && w.next(sb, g0, g1)) {
+        if (!mbar_wait(bar(B_QE), (seg & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(bar(B_QF), Q_BYTES);
+        for (int ch = 0; ch < Q_SMEM_CHUNKS; ++ch)
+          tma_load_2d(base + OFF_Q + ch * Q_CHUNK_BYTES, &tm_q, bar(B_QF), ch * 64, sb * HQ);
+        q_last = seg;
+        const int32_t* row = a.block_table + (size_t)sb * a.max_pages;
+        for (int gp = g0; gp < g1; ++gp, ++g) {
+          int page = row[gp - pref[sb]];
+          if (page < 0 || page >= a.num_pages) {
+            atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
+            page = 0;   // never read outside the pool; the result of this sequence is undefined
+          }
+          const int st = g % STAGES;
+          if (!mbar_wait(bar(B_KE + st), ((g / STAGES) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(B_KF + st), STAGE_BYTES);
+          for (int ch = 0; ch < CHUNKS; ++ch)
+            tma_load_2d(base + OFF_KV + st * STAGE_BYTES + ch * PAGE_CHUNK_BYTES, &tm_kv, bar(B_KF + st), ch * 64,
+                         page * PAGE);
+          ++issued;
+        }
+        ++seg;
+      }
+      for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait_drain(bar(B_KF + j % STAGES), (j / STAGES) & 1);
+      if (q_last >= 0) mbar_wait_drain(bar(B_QF), q_last & 1);
+    }
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
+      SegWalk w;
+      w.init(pref, a.B, R0, R1);
+      int sb, g0, g1, seg = 0, g = 0;
+      bool ok = true;
+      auto issue_pv = [&](int gp, bool first) -> bool {
+        if (!mbar_wait(bar(B_PF), gp & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const int st = gp % STAGES;
+        const uint32_t vb = base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < PAGE / 16; ++kk)
+          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, sdesc_sw128(vb + kk * 16 * 128, PAGE_CHUNK_BYTES, 1024),
+                 idesc_o, (first && kk == 0) ? 0u : 1u);
+        mma_commit(bar(B_OD));
+        mma_commit(bar(B_KE + st));
+        return true;
+      };
+      while (ok && w.next(sb, g0, g1)) {
+        if (!mbar_wait(bar(B_QF), seg & 1, abort_flag, a.status)) break;
+        if (!mbar_wait(bar(B_QT), seg & 1, abort_flag, a.status)) break;
+        for (int gp = g0; gp < g1; ++gp, ++g) {
+          const int st = g % STAGES;
+          if (!mbar_wait(bar(B_KF + st), (g / STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (g > 0 && !mbar_wait(bar(B_SE), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = base + OFF_KV + st * STAGE_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < DK / 16; ++ks) {
+            const uint64_t bdesc = sdesc_sw128(kb + (ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32, 16, 1024);
+            if (ks < Q_SMEM_CHUNKS * 4) {
+              const uint64_t adesc = sdesc_sw128(base + OFF_Q + (ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32, 16, 1024);
+              mma_ss(tmem + S_COL, adesc, bdesc, idesc_s, ks > 0);
+            } else {
+              mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, bdesc, idesc_s, 1u);
+            }
+          }
+          mma_commit(bar(B_SF));
+          if (gp == g1 - 1) mma_commit(bar(B_QE));   // last score tile of the segment: Q may be replaced
+          if (gp > g0) {
+            if (!issue_pv(g - 1, gp - 1 == g0)) { ok = false; break; }
+          } else if (seg > 0) {
+            // the previous segment's epilogue must have read O before it is overwritten
+            if (!mbar_wait(bar(B_OF), (seg - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          }
+        }
+        if (!ok) break;
+        if (!issue_pv(g - 1, g1 - 1 == g0)) break;
+        ++seg;
+      }
+      mma_commit(bar(B_DR));
+      mbar_wait_drain(bar(B_DR), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax (thread = head)
+    const int h = warp * 32 + lane;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const uint32_t t_row = tmem + lane_off;
+    const float sl2 = a.scale_log2;
+    SegWalk w;
+    w.init(pref, a.B, R0, R1);
+    int sb, g0, g1, seg = 0, g = 0;
+    bool ok = true;
+    while (ok && w.next(sb, g0, g1)) {
+      // Q dims 256..575 of this head into TMEM (the previous segment's score
+      // MMAs are complete: its epilogue waited for its last P V product).
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)sb * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
+#pragma unroll
+        for (int c = 0; c < Q_TMEM_DIMS / 64; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 u = __ldg(src + c * 8 + i);
+            r[4 * i] = u.x;
+            r[4 * i + 1] = u.y;
+            r[4 * i + 2] = u.z;
+            r[4 * i + 3] = u.w;
+          }
+          tmem_st32(t_row + Q_COL + c * 32, r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_QT));
+      }
+      const int L = seq_len_eff(a.seqlens[sb], a.max_pages);
+      const int first_page = pref[sb];
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int gp = g0; gp < g1; ++gp, ++g) {
+        if (!warp_wait(bar(B_SF), g & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t s[PAGE];
+        tmem_ld32(t_row + S_COL, s);
+        tmem_ld32(t_row + S_COL + 32, s + 32);
+        tmem_ld_wait();
+        reg_fence32(s);
+        reg_fence32(s + 32);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SE));   // S may be overwritten by the next page's scores
+        const int valid = L - (gp - first_page) * PAGE;   // tokens of this page inside the sequence
+        if (valid < PAGE) {
+#pragma unroll
+          for (int c = 0; c < PAGE; ++c)
+            if (c >= valid) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < PAGE; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool grow = m_new > m_run + kRescaleThreshold;
+        const float m_use = grow ? m_new : m_run;
+        const float alpha = grow ? ex2(m_run - m_use) : 1.f;
+        const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t p[PAGE / 2];
+#pragma unroll
+        for (int c = 0; c < PAGE / 2; ++c) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_eff));
+          const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_eff));
+          sum0 += p0;
+          sum1 += p1;
+          p[c] = pack_bf16x2(p0, p1);
+        }
+        l_run = l_run * alpha + (sum0 + sum1);
+        m_run = m_use;
+        if (gp > g0) {
+          // the previous page's P V product must be complete before P and O change
+          if (!warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (__any_sync(0xffffffffu, grow)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 256 / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_row + O_COL + c * 32, o);
+              tmem_ld_wait();
+              reg_fence32(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(t_row + O_COL + c * 32, o);
+            }
+          }
+        }
+        tmem_st32(t_row + P_COL, p);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PF));
+      }
+      if (!ok) break;
+      // -------------------------------------------------------- segment epilogue
+      if (!warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const bool full = (g0 == pref[sb]) && (g1 == pref[sb + 1]);
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float lse = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      int slot = 2 * pair + (g0 == R0 ? 0 : 1);
+#pragma unroll 1
+      for (int c = 0; c < 256 / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_row + O_COL + c * 32, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+        const int col = half * 256 + c * 32;
+        if (full) {
+          uint4* dst = reinterpret_cast<uint4*>(a.o + ((size_t)sb * HQ + h) * DV + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+            dst[i] = u;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.ws_o + ((size_t)slot * HQ + h) * DV + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                 __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+        }
+      }
+      if (half == 0) {
+        if (full) a.lse[(size_t)sb * HQ + h] = lse;
+        else a.ws_lse[(size_t)slot * HQ + h] = lse;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_OF));   // O may be overwritten by the next segment
+      ++seg;
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// One CTA per (sequence, group of 16 heads): merges the partial results of a
+// sequence that several CTA pairs shared; writes O = 0, LSE = -inf for an
+// empty sequence; leaves sequences written by the split kernel untouched.
+constexpr int COMBINE_HEADS = 16;
+constexpr int COMBINE_THREADS = 256;
+constexpr int MAX_PARTS = 128;   // >= CTA pairs, so a sequence never has more pieces
+
+__global__ void __launch_bounds__(COMBINE_THREADS)
+    decode_combine_kernel(const Args a) {
+  const int b = blockIdx.x;
+  const int h0 = blockIdx.y * COMBINE_HEADS;
+  const int tid = threadIdx.x;
+  const int T = a.ws_pref[a.B];
+  const int s0 = a.ws_pref[b], s1 = a.ws_pref[b + 1];
+  if (s1 == s0) {
+    for (int i = tid; i < COMBINE_HEADS * DV; i += COMBINE_THREADS)
+      a.o[((size_t)b * HQ + h0) * DV + i] = __float2bfloat16(0.f);
+    if (tid < COMBINE_HEADS) a.lse[(size_t)b * HQ + h0 + tid] = -INFINITY;
+    return;
+  }
+  const int p_lo = pair_of_page(s0, T, a.pairs), p_hi = pair_of_page(s1 - 1, T, a.pairs);
+  if (p_lo == p_hi) return;
+  __shared__ float w_s[COMBINE_HEADS][MAX_PARTS];
+  __shared__ int slot_s[MAX_PARTS];
+  __shared__ int nparts_s;
+  if (tid == 0) {
+    // pairs with an empty range (fewer pages than pairs) hold no piece
+    int n = 0;
+    for (int p = p_lo; p <= p_hi && n < MAX_PARTS; ++p) {
+      const int r0 = range_start(p, T, a.pairs);
+      if (range_start(p + 1, T, a.pairs) == r0) continue;
+      slot_s[n++] = 2 * p + ((p == p_lo && s0 != r0) ? 1 : 0);
+    }
+    nparts_s = n;
+  }
+  __syncthreads();
+  const int nparts = nparts_s;
+  if (tid < COMBINE_HEADS) {
+    const int h = h0 + tid;
+    float mx = -INFINITY;
+    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) mx = fmaxf(mx, a.ws_lse[(size_t)slot_s[i] * HQ + h]);
+    float sum = 0.f;
+    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) {
+      const float e = (mx == -INFINITY) ? 0.f : expf(a.ws_lse[(size_t)slot_s[i] * HQ + h] - mx);
+      w_s[tid][i] = e;
+      sum += e;
+    }
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) w_s[tid][i] *= inv;
+    a.lse[(size_t)b * HQ + h] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+  }
+  __syncthreads();
+  // 16 heads x 512 columns, 4 columns per thread per step
+  for (int i = tid; i < COMBINE_HEADS * DV / 4; i += COMBINE_THREADS) {
+    const int hh = i / (DV / 4), c4 = i % (DV / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < nparts && j < MAX_PARTS; ++j) {
+      const float wgt = w_s[hh][j];
+      const float4 v = *reinterpret_cast<const float4*>(a.ws_o + ((size_t)slot_s[j] * HQ + h0 + hh) * DV + c4 * 4);
+      acc.x += wgt * v.x;
+      acc.y += wgt * v.y;
+      acc.z += wgt * v.z;
+      acc.w += wgt * v.w;
+    }
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh) * DV + c4 * 4);
+    dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+    dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+  }
+}
+
+struct WsLayout {
+  size_t off_pref, off_lse, off_o, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(int B, int pairs) {
+  WsLayout w;
+  w.off_pref = 0;
+  w.off_lse = align256((size_t)(B + 1) * 4);
+  w.off_o = w.off_lse + align256((size_t)2 * pairs * HQ * 4);
+  w.total = w.off_o + (size_t)2 * pairs * HQ * DV * 4;
+  return w;
+}
+
+inline int pairs_for_device() {
+  const int sms = current_sm_count();
+  return sms >= 2 ? sms / 2 : 0;
+}
+
+}  // namespace dec
+}  // namespace ea
 
 extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv) {
-  (void)B;
-  (void)Hq;
-  (void)Dv;
-  return 0;
+  using namespace ea::dec;
+  if (B < 1 || B > B_MAX || Hq != HQ || Dv != DV) return 0;
+  const int pairs = pairs_for_device();
+  if (pairs == 0) return 0;
+  return ws_layout(B, pairs).total;
 }
 
 extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_table,
                                  const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk, int Dv,
                                  int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  return ATTN_ERR_UNSUPPORTED;
+  using namespace ea;
+  using namespace ea::dec;
+  if (!q || !kv_pages || !block_table || !cache_seqlens || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv_pages, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(block_table, 4) || !aligned(cache_seqlens, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || num_pages < 1 || max_pages_per_seq < 1 || page_size < 1 || Hq < 1 || Dk < 1 || Dv < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (Hq != HQ || Dk != DK || Dv != DV || page_size != PAGE || B > B_MAX) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)num_pages * PAGE >= (1ll << 31) || (long long)B * max_pages_per_seq >= (1ll << 31))
+    return ATTN_ERR_UNSUPPORTED;
+  const int pairs = pairs_for_device();
+  if (pairs == 0) return ATTN_ERR_CUDA;
+  if (pairs > MAX_PARTS) return ATTN_ERR_UNSUPPORTED;
+  const WsLayout wl = ws_layout(B, pairs);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
+
+  static int attr_done = 0;
+  if (int rc = ensure_smem_attr(reinterpret_cast<const void*>(&decode_split_kernel), SMEM_BYTES, &attr_done))
+    return rc;
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+
+  CUtensorMap tq, tkv;
+  {
+    const uint64_t dims[2] = {(uint64_t)DK, (uint64_t)B * HQ};
+    const uint64_t strides[1] = {(uint64_t)DK * 2};
+    const uint32_t box[2] = {64, (uint32_t)HQ};
+    if (!encode_bf16_2d(&tq, q, dims, strides, box)) return ATTN_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)DK, (uint64_t)num_pages * PAGE};
+    const uint64_t strides[1] = {(uint64_t)DK * 2};
+    const uint32_t box[2] = {64, (uint32_t)PAGE};
+    if (!encode_bf16_2d(&tkv, kv_pages, dims, strides, box)) return ATTN_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Args a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.block_table = block_table;
+  a.seqlens = cache_seqlens;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.ws_pref = reinterpret_cast<int32_t*>(ws + wl.off_pref);
+  a.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
+  a.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
+  a.status = status;
+  a.B = B;
+  a.max_pages = max_pages_per_seq;
+  a.num_pages = num_pages;
+  a.pairs = pairs;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  decode_split_kernel<<<2 * pairs, THREADS, SMEM_BYTES, s>>>(tq, tkv, a);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  decode_combine_kernel<<<dim3(B, HQ / COMBINE_HEADS), COMBINE_THREADS, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

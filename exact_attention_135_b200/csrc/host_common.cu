@@ -80,6 +80,11 @@ bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], 
   return encode_bf16(map, base, 4, dims, strides, box);
 }
 
+bool encode_bf16_2d(CUtensorMap* map, const void* base, const uint64_t dims[2], const uint64_t strides[1],
+                    const uint32_t box[2]) {
+  return encode_bf16(map, base, 2, dims, strides, box);
+}
+
 bool encode_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
                     const uint32_t box[3]) {
   return encode_bf16(map, base, 3, dims, strides, box);
