@@ -19,8 +19,8 @@ import re
 
 import torch
 
-__all__ = ["fwd", "decode_paged", "decode_workspace_size", "read_device_status", "library", "AttnError",
-           "exported_symbols", "STATUS"]
+__all__ = ["fwd", "decode_paged", "decode_paged_noalloc", "decode_workspace_size", "read_device_status",
+           "library", "AttnError", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libattn_b200.so")
@@ -50,6 +50,8 @@ _SIGNATURES = {
     "attn_decode_paged_workspace_size": (_sz, [_i, _i, _i]),
     "attn_decode_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_read_device_status": (_i, [_i]),
+    "attn_decode_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "attn_decode_paged_noalloc_max_bytes": (_sz, []),
 }
 
 
@@ -173,6 +175,35 @@ def decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Ten
                                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                          _stream_handle(q.device))
     _check(rc, "attn_decode_paged")
+    return out, lse
+
+
+def decode_paged_noalloc(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Tensor,
+                         cache_seqlens: torch.Tensor, scale: float, dv: int = 512, out: torch.Tensor | None = None,
+                         lse: torch.Tensor | None = None):
+    """decode_paged for callers that cannot allocate a workspace: the library
+    uses its own fixed scratch array (shared by all calls; calls that overlap
+    on the GPU race).  Outputs are allocated here only when not given."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kv_pages, "kv_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    B, sq, Hq, Dk = q.shape
+    num_pages, page_size, hkv, Dk2 = kv_pages.shape
+    if sq != 1 or hkv != 1 or Dk2 != Dk or block_table.shape[0] != B or cache_seqlens.shape[0] != B:
+        raise ValueError("decode_paged_noalloc shape mismatch")
+    if out is None:
+        out = torch.empty((B, 1, Hq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 2)
+    with torch.cuda.device(q.device):
+        rc = library().attn_decode_paged_noalloc(q.data_ptr(), kv_pages.data_ptr(), block_table.data_ptr(),
+                                                 cache_seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq,
+                                                 Dk, dv, page_size, num_pages, block_table.shape[1], float(scale),
+                                                 _stream_handle(q.device))
+    _check(rc, "attn_decode_paged_noalloc")
     return out, lse
 
 

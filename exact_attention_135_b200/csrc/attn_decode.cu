@@ -27,6 +27,8 @@
 // pages (2 x 72 KB).
 #include <math.h>
 
+#include <mutex>
+
 #include "host_common.h"
 #include "sm100.cuh"
 
@@ -623,4 +625,65 @@ extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int3
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<<<dim3(B, HQ / COMBINE_HEADS), COMBINE_THREADS, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of attn_decode_paged.
+//
+// Some callers cannot allocate device memory when they decode: a serving
+// engine that hands the whole of HBM to its own KV-cache pool at start-up has
+// no spare allocation to give a per-call workspace, and latency-critical
+// decode loops are often not allowed to call the CUDA allocator at all.  For
+// them the split-KV workspace lives in a fixed array of this library instead.
+//
+// The array below is a host-side stand-in in host code, not a device
+// address: its device address is looked up once per device (with that device
+// current) and cached.  The first call on each device performs that lookup,
+// so make the first call on a device before any stream capture.  Every GPU
+// that loads this library holds the array (kNoAllocScratchBytes) until the
+// process exits.  All calls share it and it keeps the last call's contents:
+// nothing in it has to start at zero (every value the kernels read is written
+// earlier in the same call), but calls whose kernels overlap on the GPU (two
+// streams, or two threads) race on it and must be serialised by the caller.
+namespace ea {
+namespace dec {
+
+constexpr size_t kNoAllocScratchBytes = size_t(40) << 20;   // 40 MiB
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device, or nullptr.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress((void**)&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+}  // namespace dec
+}  // namespace ea
+
+extern "C" size_t attn_decode_paged_noalloc_max_bytes(void) { return ea::dec::kNoAllocScratchBytes; }
+
+extern "C" int attn_decode_paged_noalloc(const void* q, const void* kv_pages, const int32_t* block_table,
+                                         const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk,
+                                         int Dv, int page_size, int num_pages, int max_pages_per_seq, float scale,
+                                         void* stream) {
+  using namespace ea::dec;
+  const size_t need = attn_decode_paged_workspace_size(B, Hq, Dv);
+  if (need > kNoAllocScratchBytes) return ATTN_ERR_UNSUPPORTED;   // batch too large for the fixed array
+  void* scratch = noalloc_scratch();
+  if (!scratch) return ATTN_ERR_CUDA;
+  return attn_decode_paged(q, kv_pages, block_table, cache_seqlens, o, lse, B, Hq, Dk, Dv, page_size, num_pages,
+                           max_pages_per_seq, scale, scratch, kNoAllocScratchBytes, stream);
 }

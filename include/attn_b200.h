@@ -124,6 +124,32 @@ int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_
                       size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_paged_noalloc: attn_decode_paged without a caller workspace.
+ * The source pages describe no counterpart of this entry point; it exists for
+ * callers that cannot allocate device memory at decode time (a serving engine
+ * that gives all of HBM to its own KV-cache pool has no room for a per-call
+ * workspace, and latency-critical decode loops may not call the allocator).
+ *
+ * Arguments, layouts, results and errors are those of attn_decode_paged.  The
+ * split-KV scratch is a fixed array inside this library of
+ * attn_decode_paged_noalloc_max_bytes() bytes (40 MiB), held on every GPU
+ * that loads the library until the process exits; a batch whose workspace
+ * (attn_decode_paged_workspace_size) exceeds it is rejected with
+ * ATTN_ERR_UNSUPPORTED before anything is enqueued.  The call allocates no
+ * device memory.  The first call on each device looks up the array's device
+ * address (with that device current), so make it before any stream capture.
+ * All calls share the array and it keeps the last call's contents: calls whose
+ * kernels overlap on the GPU (several streams or threads) race on it and must
+ * be serialised by the caller.
+ */
+int attn_decode_paged_noalloc(const void* q, const void* kv_pages, const int32_t* block_table,
+                              const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk, int Dv,
+                              int page_size, int num_pages, int max_pages_per_seq, float scale, void* stream);
+
+/* Size in bytes of the fixed scratch array used by attn_decode_paged_noalloc. */
+size_t attn_decode_paged_noalloc_max_bytes(void);
+
+/*
  * attn_read_device_status: status recorded by kernels on `device` since the
  * last call (ATTN_OK if none), then reset to ATTN_OK.  Synchronises with the
  * device first.  Returns ATTN_ERR_CUDA if the device cannot be queried.
