@@ -28,24 +28,38 @@
 
 namespace ea {
 
-template <int D_, bool CAUSAL_>
+template <int D_, bool CAUSAL_, int BN_>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr bool CAUSAL = CAUSAL_;
   static constexpr int BM = 128;                     // query rows per tile = TMEM lanes
   static constexpr int NT = (D <= 128) ? 2 : 1;      // Q tiles per CTA
-  static constexpr int BN = (D <= 128) ? 128 : 64;   // keys per block
-  static constexpr int NSL = 2 / NT;                 // S buffers per tile
-  static constexpr int STAGES = (D == 64) ? 3 : 2;   // K/V ring depth
+  static constexpr int BN = BN_;                     // keys per block
+  // S buffers per tile: two whenever they fit next to O in the tile's 256
+  // TMEM columns, so S of block j+1 overlaps the softmax of block j.
+  static constexpr int NSL = (NT == 1 || 2 * BN + D <= 256) ? 2 : 1;
+  static constexpr int KV_TILE = BN * D * 2;
+  static constexpr int KV_BUDGET = 224 * 1024 - NT * BM * D * 2;      // shared memory left for K/V
+  static constexpr int KSTAGES = (KV_BUDGET / KV_TILE + 1) / 2;      // K ring (released after S)
+  static constexpr int VSTAGES = KV_BUDGET / KV_TILE - KSTAGES;      // V ring (held until P V)
   static constexpr int DCH = D / 64;                 // 128-byte column chunks
   static constexpr int Q_CHUNK = BM * 128;           // bytes of one chunk of a Q tile
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int SOFTMAX_WARPS = 4 * NT;
-  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // Q and K loads
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
-  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+  static constexpr int V_PRODUCER_WARP = SOFTMAX_WARPS + 2;  // V loads, never queued behind K
+  // The three issuing warps plus one idle warp form a full warpgroup, so the
+  // register budget can move from it to the softmax warpgroups.
+  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
+  static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
+  static constexpr int ISSUE_REGS = 56;
+  static constexpr int SOFTMAX_REGS =
+      ((65536 - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8 > 248
+          ? 248
+          : ((65536 - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8;
   // TMEM columns: tile t owns [t*TILE_COLS, ...): NSL S buffers of BN
   // columns, then O (D columns).
   static constexpr int TILE_COLS = 256;
@@ -54,10 +68,10 @@ struct FwdCfg {
   // barriers
   static constexpr int B_QF = 0;
   static constexpr int B_KF = B_QF + NT;
-  static constexpr int B_KE = B_KF + STAGES;
-  static constexpr int B_VF = B_KE + STAGES;
-  static constexpr int B_VE = B_VF + STAGES;
-  static constexpr int B_SF = B_VE + STAGES;
+  static constexpr int B_KE = B_KF + KSTAGES;
+  static constexpr int B_VF = B_KE + KSTAGES;
+  static constexpr int B_VE = B_VF + VSTAGES;
+  static constexpr int B_SF = B_VE + VSTAGES;
   static constexpr int B_PF = B_SF + NT * NSL;
   static constexpr int B_OD = B_PF + NT;
   static constexpr int B_DR = B_OD + NT;
@@ -65,8 +79,8 @@ struct FwdCfg {
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * KV_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -85,12 +99,62 @@ struct FwdArgs {
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Max of the N raw scores of one row (four independent three-input chains).
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t* s) {
+  float m0 = __uint_as_float(s[0]), m1 = __uint_as_float(s[1]);
+  float m2 = __uint_as_float(s[2]), m3 = __uint_as_float(s[3]);
+#pragma unroll
+  for (int c = 4; c + 8 <= N; c += 8) {
+    m0 = max3f(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+    m1 = max3f(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+    m2 = max3f(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+    m3 = max3f(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+  }
+  m0 = max3f(m0, __uint_as_float(s[N - 4]), __uint_as_float(s[N - 3]));
+  m1 = max3f(m1, __uint_as_float(s[N - 2]), __uint_as_float(s[N - 1]));
+  return fmaxf(max3f(m0, m1, m2), m3);
+}
+
+// Pairs of columns whose exp2 runs on the FMA pipe in full blocks: 5 of every
+// 16 pairs, which balances the MUFU unit against the issue slots the
+// polynomial costs.
+__device__ __forceinline__ constexpr bool poly_pair(int c) { return (c & 15) >= 11; }
+
+// p = 2^(s * sl2 - m) for one row, packed to bf16 pairs; returns the fp32 sum.
+template <int N, bool MIXED>
+__device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float sl2, float m) {
+  const uint64_t k2 = f2_pack(sl2, sl2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int c = 0; c < N / 2; ++c) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), k2, nm2);
+    float p0, p1;
+    if (MIXED && poly_pair(c)) {
+      exp2_poly_x2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    if (c & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
+    else acc0 = f2_add(acc0, f2_pack(p0, p1));
+    p[c] = pack_bf16x2(p0, p1);
+  }
+  float a0, a1, b0, b1;
+  f2_unpack(acc0, a0, a1);
+  f2_unpack(acc1, b0, b1);
+  return (a0 + b0) + (a1 + b1);
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdArgs a) {
-  constexpr int NT = C::NT, BN = C::BN, NSL = C::NSL, ST = C::STAGES, D = C::D;
+  constexpr int NT = C::NT, BN = C::BN, NSL = C::NSL, KST = C::KSTAGES, VST = C::VSTAGES, D = C::D;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -127,9 +191,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
     for (int t = 0; t < NT; ++t) mbar_init(bar(C::B_QF + t), 1);
 #pragma unroll
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(bar(C::B_KF + s), 1);
       mbar_init(bar(C::B_KE + s), 1);
+    }
+#pragma unroll
+    for (int s = 0; s < VST; ++s) {
       mbar_init(bar(C::B_VF + s), 1);
       mbar_init(bar(C::B_VE + s), 1);
     }
@@ -158,7 +225,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= C::SOFTMAX_WARPS) {
+    // ============================================================ issue warpgroup
+    if constexpr (C::NT == 2) regs_decrease<C::ISSUE_REGS>();
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -173,18 +242,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         r0, b);
         }
       }
-      int k_issued = 0, v_issued = 0;
+      int k_issued = 0;
       for (int j = 0; j < nmax; ++j) {
-        const int st = j % ST;
-        const uint32_t ph = (j / ST) & 1;
-        if (!mbar_wait(bar(C::B_KE + st), ph ^ 1, abort_flag, a.status)) break;
+        const int st = j % KST;
+        if (!mbar_wait(bar(C::B_KE + st), ((j / KST) & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
           tma_load_4d(base + C::OFF_K + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_k, bar(C::B_KF + st), ch * 64, hk,
                       j * BN, b);
         ++k_issued;
-        if (!mbar_wait(bar(C::B_VE + st), ph ^ 1, abort_flag, a.status)) break;
+      }
+      // Drain: every issued copy must land before shared memory is released.
+      for (int j = max(0, k_issued - KST); j < k_issued; ++j) mbar_wait_drain(bar(C::B_KF + j % KST), (j / KST) & 1);
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        if (nblk[t] > 0) mbar_wait_drain(bar(C::B_QF + t), 0);
+    }
+    __syncwarp();
+  } else if (warp == C::V_PRODUCER_WARP) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      int v_issued = 0;
+      for (int j = 0; j < nmax; ++j) {
+        const int st = j % VST;
+        if (!mbar_wait(bar(C::B_VE + st), ((j / VST) & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(bar(C::B_VF + st), C::KV_BYTES);
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
@@ -192,86 +274,91 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       j * BN, b);
         ++v_issued;
       }
-      // Drain: every issued copy must land before shared memory is released.
-      for (int j = max(0, k_issued - ST); j < k_issued; ++j) mbar_wait_drain(bar(C::B_KF + j % ST), (j / ST) & 1);
-      for (int j = max(0, v_issued - ST); j < v_issued; ++j) mbar_wait_drain(bar(C::B_VF + j % ST), (j / ST) & 1);
-#pragma unroll
-      for (int t = 0; t < NT; ++t)
-        if (nblk[t] > 0) mbar_wait_drain(bar(C::B_QF + t), 0);
+      for (int j = max(0, v_issued - VST); j < v_issued; ++j) mbar_wait_drain(bar(C::B_VF + j % VST), (j / VST) & 1);
     }
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-      bool ok = true;
+    // The whole warp runs the schedule (descriptors stay warp-uniform); one
+    // elected lane issues each tcgen05 instruction.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+    bool ok = true;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+      if (ok && nblk[t] > 0) ok = warp_wait(bar(C::B_QF + t), 0, abort_flag, a.status);
+
+    auto last_tile = [&](int j) {
+      int lt = -1;
 #pragma unroll
       for (int t = 0; t < NT; ++t)
-        if (ok && nblk[t] > 0) ok = mbar_wait(bar(C::B_QF + t), 0, abort_flag, a.status);
-
-      auto last_tile = [&](int j) {
-        int lt = -1;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-          if (j < nblk[t]) lt = t;
-        return lt;
-      };
-      // S(t, j) = Q_t K_j^T into S buffer j % NSL of tile t.
-      auto issue_s = [&](int t, int j) -> bool {
-        const int st = j % ST;
-        if (!mbar_wait(bar(C::B_KF + st), (j / ST) & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
-        const uint32_t qa = base + C::OFF_Q + t * C::Q_BYTES;
-        const uint32_t kb = base + C::OFF_K + st * C::KV_BYTES;
+        if (j < nblk[t]) lt = t;
+      return lt;
+    };
+    // S(t, j) = Q_t K_j^T into S buffer j % NSL of tile t.
+    auto issue_s = [&](int t, int j) -> bool {
+      const int st = j % KST;
+      if (!warp_wait(bar(C::B_KF + st), (j / KST) & 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
+      const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
+      if (leader) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off_q = (ks >> 2) * C::Q_CHUNK + (ks & 3) * 32;
-          const uint32_t off_k = (ks >> 2) * C::KV_CHUNK + (ks & 3) * 32;
-          mma_ss(d_tmem, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(kb + off_k, 16, 1024), idesc_s, ks > 0);
+          // advance the start-address field (16-byte units) to k-step ks
+          const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
+          const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
+          mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0);
         }
         mma_commit(bar(C::B_SF + t * NSL + (j % NSL)));
         if (t == last_tile(j)) mma_commit(bar(C::B_KE + st));
-        return true;
-      };
+      }
+      __syncwarp();
+      return true;
+    };
 
-      for (int i = 0; ok && i < NSL; ++i)
+    for (int i = 0; ok && i < NSL; ++i)
 #pragma unroll
-        for (int t = 0; t < NT; ++t)
-          if (ok && i < nblk[t]) ok = issue_s(t, i);
+      for (int t = 0; t < NT; ++t)
+        if (ok && i < nblk[t]) ok = issue_s(t, i);
 
-      for (int j = 0; ok && j < nmax; ++j) {
-        const int st = j % ST;
-        bool v_ready = false;
+    for (int j = 0; ok && j < nmax; ++j) {
+      const int st = j % VST;
+      bool v_ready = false;
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if (!ok || j >= nblk[t]) continue;
-          if (!mbar_wait(bar(C::B_PF + t), j & 1, abort_flag, a.status)) { ok = false; break; }
-          if (!v_ready) {
-            if (!mbar_wait(bar(C::B_VF + st), (j / ST) & 1, abort_flag, a.status)) { ok = false; break; }
-            v_ready = true;
-          }
-          tc_fence_after();
-          const uint32_t p_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
-          const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
-          const uint32_t vb = base + C::OFF_V + st * C::KV_BYTES;
+      for (int t = 0; t < NT; ++t) {
+        if (!ok || j >= nblk[t]) continue;
+        if (!warp_wait(bar(C::B_PF + t), j & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!v_ready) {
+          if (!warp_wait(bar(C::B_VF + st), (j / VST) & 1, abort_flag, a.status)) { ok = false; break; }
+          v_ready = true;
+        }
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
+        const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
+        const uint64_t vdesc = sdesc_sw128(base + C::OFF_V + st * C::KV_BYTES, C::KV_CHUNK, 1024);
+        if (leader) {
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ts(o_tmem, p_tmem + ks * 8, sdesc_sw128(vb + ks * 16 * 128, C::KV_CHUNK, 1024), idesc_o,
-                   (j > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(o_tmem, p_tmem + ks * 8, vdesc + ((ks * 16 * 128) >> 4), idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(bar(C::B_OD + t));
           if (t == last_tile(j)) mma_commit(bar(C::B_VE + st));
-          if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
         }
+        __syncwarp();
+        if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
       }
-      // Drain: no MMA may still run when TMEM is released.
-      mma_commit(bar(C::B_DR));
-      mbar_wait_drain(bar(C::B_DR), 0);
     }
+    // Drain: no MMA may still run when TMEM is released.
+    if (leader) mma_commit(bar(C::B_DR));
     __syncwarp();
+    mbar_wait_drain(bar(C::B_DR), 0);
+    __syncwarp();
+  }
   } else {
     // ------------------------------------------------------------ softmax
+    if constexpr (C::NT == 2) regs_increase<C::SOFTMAX_REGS>();
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int row_in_tile = wq * 32 + lane;
@@ -304,25 +391,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int c = 0; c < BN; ++c)
           if (c >= cl) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+      const float mx = row_max<BN>(s);
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool grow = m_new > m_run + kRescaleThreshold;
       const float m_use = grow ? m_new : m_run;
       const float alpha = grow ? ex2(m_run - m_use) : 1.f;
       const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-      float sum0 = 0.f, sum1 = 0.f;
       uint32_t p[BN / 2];
-#pragma unroll
-      for (int c = 0; c < BN / 2; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_eff));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_eff));
-        sum0 += p0;
-        sum1 += p1;
-        p[c] = pack_bf16x2(p0, p1);
-      }
-      l_run = l_run * alpha + (sum0 + sum1);
+      // Blocks with masked keys use the MUFU exp2 only (masked scores are -inf
+      // and must give exactly 0); full blocks send part of the work to the FMA pipe.
+      const float sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
+      l_run = l_run * alpha + sum;
       m_run = m_use;
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(t_tmem + slot * BN + c * 32, p + c * 32);
@@ -407,7 +486,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 template <int D, bool CAUSAL>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, cudaStream_t stream) {
-  using C = FwdCfg<D, CAUSAL>;
+  using C = FwdCfg<D, CAUSAL, (D <= 128) ? 128 : 64>;
   static int attr_done = 0;
   const void* kfn = reinterpret_cast<const void*>(&attn_fwd_kernel<C>);
   if (int rc = ensure_smem_attr(kfn, C::SMEM_BYTES, &attr_done)) return rc;

@@ -176,6 +176,29 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Move registers between warpgroups (all four warps of a warpgroup execute
+// the same instruction).  The totals must stay within the launch's budget.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// One lane of a converged warp returns true (elect.sync).  Issue loops run
+// warp-wide so descriptors stay warp-uniform; only the elected lane issues.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -254,6 +277,78 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 instructions: two lanes per instruction)
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ---- 2^x on the FMA pipe (offloads the MUFU unit)
+//
+// Cody-Waite style range reduction x = n + f, n = round(x), f in [-1/2, 1/2]
+// (rounding by adding and subtracting 1.5 * 2^23), then 2^f from a degree-3
+// polynomial that minimises the maximum relative error on [-1/2, 1/2]
+// (Remez exchange, coefficients from csrc/gen_exp2_poly.py; max relative error
+// 7.5e-5 in fp32 Horner form), and 2^n added into the exponent field.
+// Inputs are clamped to >= -125, so 2^x for x < -125 returns a value below
+// 2^-124 instead of 0: use only where no input is -inf by design.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+
+// Two lanes at once: x = (x0, x1) packed.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float& y0, float& y1) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t magic = f2_pack(kRoundMagic, kRoundMagic);
+  const uint64_t t = f2_add(xc, magic);                       // round(x) in the low mantissa bits
+  const uint64_t r = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));   // round(x), exact
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), xc);                // x - round(x), exact
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
