@@ -255,61 +255,70 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
-      SegWalk w;
-      w.init(pref, a.B, R0, R1);
-      int sb, g0, g1, seg = 0, g = 0;
-      bool ok = true;
-      auto issue_pv = [&](int gp, bool first) -> bool {
-        if (!mbar_wait(bar(B_PF), gp & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const int st = gp % STAGES;
-        const uint32_t vb = base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES;
+    // Warp-wide schedule, warp-uniform descriptors; one elected lane issues.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
+    SegWalk w;
+    w.init(pref, a.B, R0, R1);
+    int sb, g0, g1, seg = 0, g = 0;
+    bool ok = true;
+    const uint64_t qdesc = sdesc_sw128(base + OFF_Q, 16, 1024);
+    auto issue_pv = [&](int gp, bool first) -> bool {
+      if (!warp_wait(bar(B_PF), gp & 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const int st = gp % STAGES;
+      const uint64_t vdesc =
+          sdesc_sw128(base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES, PAGE_CHUNK_BYTES, 1024);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < PAGE / 16; ++kk)
-          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, sdesc_sw128(vb + kk * 16 * 128, PAGE_CHUNK_BYTES, 1024),
-                 idesc_o, (first && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
+                 (first && kk == 0) ? 0u : 1u);
         mma_commit(bar(B_OD));
         mma_commit(bar(B_KE + st));
-        return true;
-      };
-      while (ok && w.next(sb, g0, g1)) {
-        if (!mbar_wait(bar(B_QF), seg & 1, abort_flag, a.status)) break;
-        if (!mbar_wait(bar(B_QT), seg & 1, abort_flag, a.status)) break;
-        for (int gp = g0; gp < g1; ++gp, ++g) {
-          const int st = g % STAGES;
-          if (!mbar_wait(bar(B_KF + st), (g / STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
-          if (g > 0 && !mbar_wait(bar(B_SE), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = base + OFF_KV + st * STAGE_BYTES;
+      }
+      __syncwarp();
+      return true;
+    };
+    while (ok && w.next(sb, g0, g1)) {
+      if (!warp_wait(bar(B_QF), seg & 1, abort_flag, a.status)) break;
+      if (!warp_wait(bar(B_QT), seg & 1, abort_flag, a.status)) break;
+      for (int gp = g0; gp < g1; ++gp, ++g) {
+        const int st = g % STAGES;
+        if (!warp_wait(bar(B_KF + st), (g / STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        if (g > 0 && !warp_wait(bar(B_SE), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t kdesc = sdesc_sw128(base + OFF_KV + st * STAGE_BYTES, 16, 1024);
+        if (leader) {
 #pragma unroll
           for (int ks = 0; ks < DK / 16; ++ks) {
-            const uint64_t bdesc = sdesc_sw128(kb + (ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32, 16, 1024);
+            const uint32_t dk = ((ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32) >> 4;
             if (ks < Q_SMEM_CHUNKS * 4) {
-              const uint64_t adesc = sdesc_sw128(base + OFF_Q + (ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32, 16, 1024);
-              mma_ss(tmem + S_COL, adesc, bdesc, idesc_s, ks > 0);
+              const uint32_t dq = ((ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32) >> 4;
+              mma_ss(tmem + S_COL, qdesc + dq, kdesc + dk, idesc_s, ks > 0);
             } else {
-              mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, bdesc, idesc_s, 1u);
+              mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, kdesc + dk, idesc_s, 1u);
             }
           }
           mma_commit(bar(B_SF));
           if (gp == g1 - 1) mma_commit(bar(B_QE));   // last score tile of the segment: Q may be replaced
-          if (gp > g0) {
-            if (!issue_pv(g - 1, gp - 1 == g0)) { ok = false; break; }
-          } else if (seg > 0) {
-            // the previous segment's epilogue must have read O before it is overwritten
-            if (!mbar_wait(bar(B_OF), (seg - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          }
         }
-        if (!ok) break;
-        if (!issue_pv(g - 1, g1 - 1 == g0)) break;
-        ++seg;
+        __syncwarp();
+        if (gp > g0) {
+          if (!issue_pv(g - 1, gp - 1 == g0)) { ok = false; break; }
+        } else if (seg > 0) {
+          // the previous segment's epilogue must have read O before it is overwritten
+          if (!warp_wait(bar(B_OF), (seg - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        }
       }
-      mma_commit(bar(B_DR));
-      mbar_wait_drain(bar(B_DR), 0);
+      if (!ok) break;
+      if (!issue_pv(g - 1, g1 - 1 == g0)) break;
+      ++seg;
     }
+    if (leader) mma_commit(bar(B_DR));
+    __syncwarp();
+    mbar_wait_drain(bar(B_DR), 0);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (thread = head)
@@ -351,11 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!warp_wait(bar(B_SF), g & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[PAGE];
-        tmem_ld32(t_row + S_COL, s);
-        tmem_ld32(t_row + S_COL + 32, s + 32);
-        tmem_ld_wait();
-        reg_fence32(s);
-        reg_fence32(s + 32);
+        tmem_ld64_sync(t_row + S_COL, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_SE));   // S may be overwritten by the next page's scores
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < PAGE; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int c = 0; c < PAGE; c += 2) mx = max3f(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = m_new > m_run + kRescaleThreshold;
         const float m_use = grow ? m_new : m_run;
@@ -393,9 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
             for (int c = 0; c < 256 / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32(t_row + O_COL + c * 32, o);
-              tmem_ld_wait();
-              reg_fence32(o);
+              tmem_ld32_sync(t_row + O_COL + c * 32, o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
               tmem_st32(t_row + O_COL + c * 32, o);
@@ -419,9 +422,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < 256 / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(t_row + O_COL + c * 32, o);
-        tmem_ld_wait();
-        reg_fence32(o);
+        tmem_ld32_sync(t_row + O_COL + c * 32, o);
         const int col = half * 256 + c * 32;
         if (full) {
           uint4* dst = reinterpret_cast<uint4*>(a.o + ((size_t)sb * HQ + h) * DV + col);

@@ -378,11 +378,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!warp_wait(bar(C::B_SF + t * NSL + slot), (j / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_tmem + slot * BN + c * 32, s + c * 32);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) reg_fence32(s + c * 32);
+if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
+      else tmem_ld64_sync(t_tmem + slot * BN, s);
 
       const bool need_mask = ((j + 1) * BN > a.Nk) || (C::CAUSAL && (j + 1) * BN - 1 > r0 + a.causal_off);
       if (need_mask) {
@@ -415,9 +412,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(t_tmem + C::O_COL + c * 32, o);
-            tmem_ld_wait();
-            reg_fence32(o);
+            tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(t_tmem + C::O_COL + c * 32, o);
@@ -443,9 +438,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         if (n > 0) {
-          tmem_ld32(t_tmem + C::O_COL + c * 32, o);
-          tmem_ld_wait();
-          reg_fence32(o);
+          tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
