@@ -64,6 +64,25 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of `values` over all ranks (identity with one rank).
+
+    Every rank must call it with a list of the same length; works for any
+    torch.distributed backend (NCCL with a CUDA device, gloo on the CPU).
+    """
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(world: int, work_per_rank: float, slowest_ms: float) -> float:
+    """Work done by all ranks together per second, timed by the slowest rank."""
+    return world * work_per_rank / (slowest_ms * 1e-3)
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -263,10 +282,7 @@ def run_gpu(args):
     names = [p.name for p in parts]
     vec = [total_ms / args.steps] + [statistics.mean(per[n]) for n in names] + \
           [statistics.mean(e2e[n]) for n in names]
-    if world > 1:
-        t = torch.tensor(vec, device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        vec = t.tolist()
+    vec = max_over_ranks(vec, device=dev)
     step_ms = vec[0]
     launch_ms = dict(zip(names, vec[1:1 + len(names)]))
     e2e_ms = dict(zip(names, vec[1 + len(names):]))
@@ -282,7 +298,8 @@ def run_gpu(args):
         p = by["decode"]
         gbs = p.kv_bytes / (launch_ms["decode"] * 1e-3) / 1e9
         decode_obj = {
-            "metric": "KV-cache GB/s (paged decode)", "value": round(world * gbs, 1), "unit": "GB/s",
+            "metric": "KV-cache GB/s (paged decode)",
+            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["decode"]) / 1e9, 1), "unit": "GB/s",
             "ms_per_launch": round(launch_ms["decode"], 4),
             "config": {"workload": p.cfg.name, "B": p.cfg.B, "Hq": p.cfg.Hq, "Dk": p.cfg.Dk, "Dv": p.cfg.Dv,
                        "page_size": p.cfg.page_size, "lengths": f"uniform [{p.cfg.min_len}, {p.cfg.max_len}]",
@@ -305,7 +322,7 @@ def run_gpu(args):
         peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         line.update({
             "metric": "attention TFLOP/s (prefill)",
-            "value": round(world * p.work / (launch_ms["prefill"] * 1e-3) / 1e12, 2),
+            "value": round(whole_job_rate(world, p.work, launch_ms["prefill"]) / 1e12, 2),
             "unit": "TFLOP/s",
             "config": {"workload": p.cfg.name, "step": step_parts, "B": p.cfg.B, "Hq": p.cfg.Hq,
                        "Hkv": p.cfg.Hkv, "Nq": p.cfg.Nq, "Nk": p.cfg.Nk, "D": p.cfg.D, "causal": p.cfg.causal,

@@ -52,6 +52,7 @@ _SIGNATURES = {
     "attn_read_device_status": (_i, [_i]),
     "attn_decode_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_decode_paged_noalloc_max_bytes": (_sz, []),
+    "attn_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
 }
 
 

@@ -150,6 +150,18 @@ int attn_decode_paged_noalloc(const void* q, const void* kv_pages, const int32_t
 size_t attn_decode_paged_noalloc_max_bytes(void);
 
 /*
+ * attn_selftest_wait_timeout: exercise the bounded-wait failure path.  The
+ * source pages describe no counterpart; this checks this library's own
+ * failure detection.  One CTA waits on a barrier that nothing ever releases,
+ * with the same bounded wait the attention kernels use but a limit of
+ * `limit_us` microseconds (1 .. 10,000,000).  When the limit passes, the kernel
+ * records ATTN_ERR_TIMEOUT in the device status word and returns normally:
+ * nothing faults or hangs and the context stays usable.  Enqueues on
+ * `stream`; read the outcome with attn_read_device_status.
+ */
+int attn_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+/*
  * attn_read_device_status: status recorded by kernels on `device` since the
  * last call (ATTN_OK if none), then reset to ATTN_OK.  Synchronises with the
  * device first.  Returns ATTN_ERR_CUDA if the device cannot be queried.

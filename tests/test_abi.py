@@ -67,3 +67,8 @@ def test_fwd_no_keys_accepts_null_kv_and_empty_query(lib):
     assert _fwd(lib, k=None, v=None, Nq=0, Nk=0) == 0
     # Nk > 0 with null K is an argument error
     assert _fwd(lib, k=None, Nk=5) == 1
+
+
+def test_selftest_rejects_bad_limits_on_host(lib):
+    assert lib.attn_selftest_wait_timeout(0, None) == 1
+    assert lib.attn_selftest_wait_timeout(20_000_000, None) == 1
