@@ -72,9 +72,13 @@ struct FwdCfg {
   static constexpr int B_VF = B_KE + KSTAGES;
   static constexpr int B_VE = B_VF + VSTAGES;
   static constexpr int B_SF = B_VE + VSTAGES;
+  // P ready, one per (tile, S buffer): the softmax of block j+NSL cannot
+  // arrive before the MMA warp has taken block j's phase (S_{j+NSL} is only
+  // issued after P_j V_j), so no barrier ever runs two phases ahead.
   static constexpr int B_PF = B_SF + NT * NSL;
-  static constexpr int B_OD = B_PF + NT;
-  static constexpr int B_DR = B_OD + NT;
+  static constexpr int B_OD = B_PF + NT * NSL;      // one phase per P V product of the tile
+  static constexpr int B_OF = B_OD + NT;      // single phase: the tile's last P V is done
+  static constexpr int B_DR = B_OF + NT;
   static constexpr int NBAR = B_DR + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_Q = 0;
@@ -201,11 +205,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(bar(C::B_VE + s), 1);
     }
 #pragma unroll
-    for (int i = 0; i < NT * NSL; ++i) mbar_init(bar(C::B_SF + i), 1);
+    for (int i = 0; i < NT * NSL; ++i) {
+      mbar_init(bar(C::B_SF + i), 1);
+      mbar_init(bar(C::B_PF + i), 4);   // one arrival per softmax warp
+    }
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-      mbar_init(bar(C::B_PF + t), 4);   // one arrival per softmax warp
       mbar_init(bar(C::B_OD + t), 1);
+      mbar_init(bar(C::B_OF + t), 1);
     }
     mbar_init(bar(C::B_DR), 1);
     *abort_flag = 0;
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         if (!ok || j >= nblk[t]) continue;
-        if (!warp_wait(bar(C::B_PF + t), j & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!warp_wait(bar(C::B_PF + t * NSL + j % NSL), (j / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
         if (!v_ready) {
           if (!warp_wait(bar(C::B_VF + st), (j / VST) & 1, abort_flag, a.status)) { ok = false; break; }
           v_ready = true;
@@ -344,6 +351,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int ks = 0; ks < BN / 16; ++ks)
             mma_ts(o_tmem, p_tmem + ks * 8, vdesc + ((ks * 16 * 128) >> 4), idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(bar(C::B_OD + t));
+          if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t));
           if (t == last_tile(j)) mma_commit(bar(C::B_VE + st));
         }
         __syncwarp();
@@ -403,31 +411,32 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(t_tmem + slot * BN + c * 32, p + c * 32);
       tmem_st_wait();
-      if (j > 0) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled (and every phase
-        // of this barrier is consumed in order).
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O must hold P_{j-1} V_{j-1} before it is rescaled.  The wait is
+        // unambiguous although most phases of this barrier are never waited
+        // on: S_j is done, so every P V issued before it (up to P_{j-2} V_{j-2})
+        // is done, and P_j V_j cannot start before this warp's arrival below;
+        // the barrier therefore sits at phase j-1 or j.
         if (!warp_wait(bar(C::B_OD + t), (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-        if (__any_sync(0xffffffffu, grow)) {
-          tc_fence_after();
+        tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_tmem + C::O_COL + c * 32, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_tmem + C::O_COL + c * 32, o);
         }
+        tmem_st_wait();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PF + t));
+      if (lane == 0) mbar_arrive(bar(C::B_PF + t * NSL + slot));
     }
 
     // ------------------------------------------------------------ epilogue
     if (ok && n > 0) {
-      ok = warp_wait(bar(C::B_OD + t), (n - 1) & 1, abort_flag, a.status);
+      ok = warp_wait(bar(C::B_OF + t), 0, abort_flag, a.status);
       tc_fence_after();
     }
     const bool write = ok && !*abort_flag;
