@@ -54,13 +54,14 @@ constexpr int S_COL = 256;
 constexpr int P_COL = 320;
 constexpr int Q_COL = 352;
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 192;                    // 4 softmax warps, producer, MMA
+constexpr int THREADS = 224;                    // 4 softmax warps, producer, two MMA issuers
 constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
+constexpr int MMA_S_WARP = 5;                   // score tiles S = Q K^T
+constexpr int MMA_PV_WARP = 6;                  // products O += P V
 // barriers
 constexpr int B_QF = 0, B_QE = 1, B_QT = 2, B_KF = 3, B_KE = B_KF + STAGES, B_SF = B_KE + STAGES;
-constexpr int B_SE = B_SF + 1, B_PF = B_SE + 1, B_OD = B_PF + 1, B_OF = B_OD + 1, B_DR = B_OF + 1;
-constexpr int NBAR = B_DR + 1;
+constexpr int B_SE = B_SF + 1, B_PF = B_SE + 1, B_OD = B_PF + 1, B_DR = B_OD + 1, B_DRS = B_DR + 1;
+constexpr int NBAR = B_DRS + 1;
 // shared memory
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + Q_BYTES;
@@ -171,8 +172,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bar(B_SE), 4);
     mbar_init(bar(B_PF), 4);
     mbar_init(bar(B_OD), 1);
-    mbar_init(bar(B_OF), 4);
     mbar_init(bar(B_DR), 1);
+    mbar_init(bar(B_DRS), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -253,34 +254,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (q_last >= 0) mbar_wait_drain(bar(B_QF), q_last & 1);
     }
     __syncwarp();
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    // Warp-wide schedule, warp-uniform descriptors; one elected lane issues.
+  } else if (warp == MMA_S_WARP) {
+    // ------------------------------------------------------------ score MMA issuer
+    // Two warps issue MMAs, each waiting only for what its own products need:
+    // this one S = Q K^T per page (page landed, S buffer read by the softmax),
+    // the next one O += P V (P written).  A P V product therefore never waits
+    // behind the next page's load, and it frees the page's stage as early as
+    // possible.  S, P and O occupy disjoint TMEM columns, so the two issue
+    // streams need no ordering between them beyond those barriers.
+    // Warp-uniform schedule; one elected lane issues.
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
     SegWalk w;
     w.init(pref, a.B, R0, R1);
     int sb, g0, g1, seg = 0, g = 0;
     bool ok = true;
     const uint64_t qdesc = sdesc_sw128(base + OFF_Q, 16, 1024);
-    auto issue_pv = [&](int gp, bool first) -> bool {
-      if (!warp_wait(bar(B_PF), gp & 1, abort_flag, a.status)) return false;
-      tc_fence_after();
-      const int st = gp % STAGES;
-      const uint64_t vdesc =
-          sdesc_sw128(base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES, PAGE_CHUNK_BYTES, 1024);
-      if (leader) {
-#pragma unroll
-        for (int kk = 0; kk < PAGE / 16; ++kk)
-          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
-                 (first && kk == 0) ? 0u : 1u);
-        mma_commit(bar(B_OD));
-        mma_commit(bar(B_KE + st));
-      }
-      __syncwarp();
-      return true;
-    };
     while (ok && w.next(sb, g0, g1)) {
       if (!warp_wait(bar(B_QF), seg & 1, abort_flag, a.status)) break;
       if (!warp_wait(bar(B_QT), seg & 1, abort_flag, a.status)) break;
@@ -305,16 +294,44 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (gp == g1 - 1) mma_commit(bar(B_QE));   // last score tile of the segment: Q may be replaced
         }
         __syncwarp();
-        if (gp > g0) {
-          if (!issue_pv(g - 1, gp - 1 == g0)) { ok = false; break; }
-        } else if (seg > 0) {
-          // the previous segment's epilogue must have read O before it is overwritten
-          if (!warp_wait(bar(B_OF), (seg - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-        }
       }
-      if (!ok) break;
-      if (!issue_pv(g - 1, g1 - 1 == g0)) break;
       ++seg;
+    }
+    // Drain: no MMA may still run when TMEM is released.
+    if (leader) mma_commit(bar(B_DRS));
+    __syncwarp();
+    mbar_wait_drain(bar(B_DRS), 0);
+    __syncwarp();
+  } else if (warp == MMA_PV_WARP) {
+    // ------------------------------------------------------------ P V MMA issuer
+    // The P of a segment's first page is written only after the previous
+    // segment's epilogue has read O (same softmax warps, in order), so the
+    // overwrite of O by that page's product needs no extra barrier.  S of a
+    // page is complete before its P exists, so this warp's completion of
+    // P V also means the page's stage is no longer read by any MMA.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
+    SegWalk w;
+    w.init(pref, a.B, R0, R1);
+    int sb, g0, g1, g = 0;
+    bool ok = true;
+    while (ok && w.next(sb, g0, g1)) {
+      for (int gp = g0; gp < g1; ++gp, ++g) {
+        if (!warp_wait(bar(B_PF), g & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const int st = g % STAGES;
+        const uint64_t vdesc =
+            sdesc_sw128(base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES, PAGE_CHUNK_BYTES, 1024);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < PAGE / 16; ++kk)
+            mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
+                   (gp == g0 && kk == 0) ? 0u : 1u);
+          mma_commit(bar(B_OD));
+          mma_commit(bar(B_KE + st));
+        }
+        __syncwarp();
+      }
     }
     if (leader) mma_commit(bar(B_DR));
     __syncwarp();
@@ -449,7 +466,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_OF));   // O may be overwritten by the next segment
       ++seg;
     }
     __syncwarp();
