@@ -31,6 +31,7 @@
 
 #include "host_common.h"
 #include "sm100.cuh"
+#include "softmax_row.cuh"
 
 namespace ea {
 
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // behind the next page's load, and it frees the page's stage as early as
     // possible.  S, P and O occupy disjoint TMEM columns, so the two issue
     // streams need no ordering between them beyond those barriers.
-    // Warp-uniform schedule; one elected lane issues.
+    // Warp-uniform schedule; one elected lane issues (predicated, no branch).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
     SegWalk w;
@@ -279,26 +280,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (g > 0 && !warp_wait(bar(B_SE), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint64_t kdesc = sdesc_sw128(base + OFF_KV + st * STAGE_BYTES, 16, 1024);
-        if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < DK / 16; ++ks) {
-            const uint32_t dk = ((ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32) >> 4;
-            if (ks < Q_SMEM_CHUNKS * 4) {
-              const uint32_t dq = ((ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32) >> 4;
-              mma_ss(tmem + S_COL, qdesc + dq, kdesc + dk, idesc_s, ks > 0);
-            } else {
-              mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, kdesc + dk, idesc_s, 1u);
-            }
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t dk = ((ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32) >> 4;
+          if (ks < Q_SMEM_CHUNKS * 4) {
+            const uint32_t dq = ((ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32) >> 4;
+            mma_ss(tmem + S_COL, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+          } else {
+            mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, kdesc + dk, idesc_s, 1u, leader);
           }
-          mma_commit(bar(B_SF));
-          if (gp == g1 - 1) mma_commit(bar(B_QE));   // last score tile of the segment: Q may be replaced
         }
+        mma_commit(bar(B_SF), leader);
+        if (gp == g1 - 1) mma_commit(bar(B_QE), leader);   // last score tile of the segment: Q may be replaced
         __syncwarp();
       }
       ++seg;
     }
     // Drain: no MMA may still run when TMEM is released.
-    if (leader) mma_commit(bar(B_DRS));
+    mma_commit(bar(B_DRS), leader);
     __syncwarp();
     mbar_wait_drain(bar(B_DRS), 0);
     __syncwarp();
@@ -322,18 +321,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = g % STAGES;
         const uint64_t vdesc =
             sdesc_sw128(base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES, PAGE_CHUNK_BYTES, 1024);
-        if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < PAGE / 16; ++kk)
-            mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
-                   (gp == g0 && kk == 0) ? 0u : 1u);
-          mma_commit(bar(B_OD));
-          mma_commit(bar(B_KE + st));
-        }
+        for (int kk = 0; kk < PAGE / 16; ++kk)
+          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
+                 (gp == g0 && kk == 0) ? 0u : 1u, leader);
+        mma_commit(bar(B_OD), leader);
+        mma_commit(bar(B_KE + st), leader);
         __syncwarp();
       }
     }
-    if (leader) mma_commit(bar(B_DR));
+    mma_commit(bar(B_DR), leader);
     __syncwarp();
     mbar_wait_drain(bar(B_DR), 0);
     __syncwarp();
@@ -382,30 +379,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_SE));   // S may be overwritten by the next page's scores
         const int valid = L - (gp - first_page) * PAGE;   // tokens of this page inside the sequence
-        if (valid < PAGE) {
+        const bool partial = valid < PAGE;
+        if (partial) {
 #pragma unroll
           for (int c = 0; c < PAGE; ++c)
             if (c >= valid) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < PAGE; c += 2) mx = max3f(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float mx = row_max<PAGE>(s);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = m_new > m_run + kRescaleThreshold;
         const float m_use = grow ? m_new : m_run;
         const float alpha = grow ? ex2(m_run - m_use) : 1.f;
         const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-        float sum0 = 0.f, sum1 = 0.f;
         uint32_t p[PAGE / 2];
-#pragma unroll
-        for (int c = 0; c < PAGE / 2; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_eff));
-          const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_eff));
-          sum0 += p0;
-          sum1 += p1;
-          p[c] = pack_bf16x2(p0, p1);
-        }
-        l_run = l_run * alpha + (sum0 + sum1);
+        // A page cut by the sequence end uses the MUFU exp2 only (its masked
+        // scores are -inf and must give exactly 0); full pages send part of
+        // the work to the FMA pipe.
+        const float sum = partial ? exp_row<PAGE, false>(s, p, sl2, m_eff) : exp_row<PAGE, true>(s, p, sl2, m_eff);
+        l_run = l_run * alpha + sum;
         m_run = m_use;
         if (gp > g0) {
           // the previous page's P V product must be complete before P and O change

@@ -25,6 +25,7 @@
 
 #include "host_common.h"
 #include "sm100.cuh"
+#include "softmax_row.cuh"
 
 namespace ea {
 
@@ -102,56 +103,6 @@ struct FwdArgs {
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
 constexpr float kLn2 = 0.6931471805599453f;
-
-// Max of the N raw scores of one row (four independent three-input chains).
-template <int N>
-__device__ __forceinline__ float row_max(const uint32_t* s) {
-  float m0 = __uint_as_float(s[0]), m1 = __uint_as_float(s[1]);
-  float m2 = __uint_as_float(s[2]), m3 = __uint_as_float(s[3]);
-#pragma unroll
-  for (int c = 4; c + 8 <= N; c += 8) {
-    m0 = max3f(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-    m1 = max3f(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-    m2 = max3f(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-    m3 = max3f(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-  }
-  m0 = max3f(m0, __uint_as_float(s[N - 4]), __uint_as_float(s[N - 3]));
-  m1 = max3f(m1, __uint_as_float(s[N - 2]), __uint_as_float(s[N - 1]));
-  return fmaxf(max3f(m0, m1, m2), m3);
-}
-
-// Pairs of columns whose exp2 runs on the FMA pipe in full blocks: 5 of every
-// 16 pairs, which balances the MUFU unit against the issue slots the
-// polynomial costs.
-__device__ __forceinline__ constexpr bool poly_pair(int c) { return (c & 15) >= 11; }
-
-// p = 2^(s * sl2 - m) for one row, packed to bf16 pairs; returns the fp32 sum.
-template <int N, bool MIXED>
-__device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float sl2, float m) {
-  const uint64_t k2 = f2_pack(sl2, sl2);
-  const uint64_t nm2 = f2_pack(-m, -m);
-  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-  for (int c = 0; c < N / 2; ++c) {
-    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), k2, nm2);
-    float p0, p1;
-    if (MIXED && poly_pair(c)) {
-      exp2_poly_x2(x, p0, p1);
-    } else {
-      float x0, x1;
-      f2_unpack(x, x0, x1);
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
-    if (c & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
-    else acc0 = f2_add(acc0, f2_pack(p0, p1));
-    p[c] = pack_bf16x2(p0, p1);
-  }
-  float a0, a1, b0, b1;
-  f2_unpack(acc0, a0, a1);
-  f2_unpack(acc1, b0, b1);
-  return (a0 + b0) + (a1 + b1);
-}
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
@@ -287,7 +238,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the schedule (descriptors stay warp-uniform); one
-    // elected lane issues each tcgen05 instruction.
+    // elected lane issues each tcgen05 instruction, predicated (no branch).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
@@ -311,17 +262,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint32_t d_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
       const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
       const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
-      if (leader) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          // advance the start-address field (16-byte units) to k-step ks
-          const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
-          const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
-          mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0);
-        }
-        mma_commit(bar(C::B_SF + t * NSL + (j % NSL)));
-        if (t == last_tile(j)) mma_commit(bar(C::B_KE + st));
+      for (int ks = 0; ks < D / 16; ++ks) {
+        // advance the start-address field (16-byte units) to k-step ks
+        const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
+        const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
+        mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
       }
+      mma_commit(bar(C::B_SF + t * NSL + (j % NSL)), leader);
+      if (t == last_tile(j)) mma_commit(bar(C::B_KE + st), leader);
       __syncwarp();
       return true;
     };
@@ -346,20 +295,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t p_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
         const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
         const uint64_t vdesc = sdesc_sw128(base + C::OFF_V + st * C::KV_BYTES, C::KV_CHUNK, 1024);
-        if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ts(o_tmem, p_tmem + ks * 8, vdesc + ((ks * 16 * 128) >> 4), idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(bar(C::B_OD + t));
-          if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t));
-          if (t == last_tile(j)) mma_commit(bar(C::B_VE + st));
-        }
+        for (int ks = 0; ks < BN / 16; ++ks)
+          mma_ts(o_tmem, p_tmem + ks * 8, vdesc + ((ks * 16 * 128) >> 4), idesc_o, (j > 0 || ks > 0) ? 1u : 0u,
+                 leader);
+        mma_commit(bar(C::B_OD + t), leader);
+        if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t), leader);
+        if (t == last_tile(j)) mma_commit(bar(C::B_VE + st), leader);
         __syncwarp();
         if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
       }
     }
     // Drain: no MMA may still run when TMEM is released.
-    if (leader) mma_commit(bar(C::B_DR));
+    mma_commit(bar(C::B_DR), leader);
     __syncwarp();
     mbar_wait_drain(bar(C::B_DR), 0);
     __syncwarp();
