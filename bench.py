@@ -46,8 +46,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu capture of the same launch; see profiles/.  Set to None whenever the
 # kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 202546176 + 106302720,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
-    "decode": 349258752 + 16388352,     # decode_split_kernel, MLA decode workload
+    "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
+    "decode": 349399808 + 16235008,     # decode_split_kernel, MLA decode workload
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.
