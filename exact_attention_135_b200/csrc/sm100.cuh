@@ -100,6 +100,13 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
 
 // ------------------------------------------------------------------ TMA
 
+// Ask L2 to fetch [ptr, ptr + bytes) (16-byte aligned, bytes a multiple of 16);
+// no shared memory and no completion to wait for.
+__device__ __forceinline__ void l2_prefetch(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(ptr)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
