@@ -16,6 +16,11 @@ with 1000 + workload number, then rounded to bf16):
    576-wide latent row per token (K = all 576, V = first 512), 64-token pages,
    lengths uniform on [1024, 8192], block table = a random permutation of the
    page pool, scale 1/sqrt(192).
+6. GQA-path paged decode: 64 sequences x 1 query token x 32 query heads in 8
+   groups of 4, each group reading its own expanded K and V rows (D=128) from
+   64-token pages; lengths uniform on [1024, 8192], random page permutation,
+   scale 1/sqrt(128).  The head geometry is LLaMA-3-8B's (the GQA model the
+   GQLA page converts); the pages give no decode shapes for this path.
 
 Paged-cache layout (decode): the pool holds exactly sum_b ceil(L_b/64) pages
 plus one poison page at the end.  Block-table entries past a sequence's last
@@ -160,6 +165,84 @@ def paged_decode_inputs(B, Hq, Dk, seqlens, page_size, seed, max_pages_per_seq=N
             last = int(table[b, npg - 1])
             pool[last, L % page_size:] = sentinel[last, L % page_size:]
     return PagedCache(q, pool, table, seqlens.clone(), page_size)
+
+
+@dataclass(frozen=True)
+class GqaDecodeConfig:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    page_size: int
+    min_len: int
+    max_len: int
+    scale: float
+    seed: int = 0
+
+
+GQA_DECODE_CONFIG = GqaDecodeConfig("GQA-path paged decode B64 Hq32 Hkv8 D128 page64", 64, 32, 8, 128, PAGE_SIZE,
+                                    1024, 8192, 1.0 / math.sqrt(128.0), seed=1006)
+
+
+@dataclass
+class PagedKV:
+    q: torch.Tensor              # [B, 1, Hq, D] bf16
+    k_pages: torch.Tensor        # [num_pages, page_size, Hkv, D] bf16 (last page = poison)
+    v_pages: torch.Tensor        # [num_pages, page_size, Hkv, D] bf16 (last page = poison)
+    block_table: torch.Tensor    # [B, max_pages_per_seq] int32
+    cache_seqlens: torch.Tensor  # [B] int32
+    page_size: int
+
+    @property
+    def num_pages(self) -> int:
+        return int(self.k_pages.shape[0])
+
+    def kv_valid_bytes(self) -> int:
+        """Bytes of K and V rows that belong to the sequences (what a decode step must read)."""
+        hkv, d = int(self.k_pages.shape[2]), int(self.k_pages.shape[3])
+        return int(self.cache_seqlens.to(torch.int64).sum()) * hkv * d * 2 * 2
+
+
+def paged_gqa_decode_inputs(B, Hq, Hkv, D, seqlens, page_size, seed, max_pages_per_seq=None):
+    """Build separate K and V page pools (GQA path: one expanded K and V row per
+    token and KV head) for the given sequence lengths.  Same pool, poison-page
+    and block-table conventions as paged_decode_inputs.  Returns a PagedKV."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int32).reshape(-1)
+    assert seqlens.numel() == B
+    pages_per_seq = [(int(L) + page_size - 1) // page_size for L in seqlens.tolist()]
+    n_used = sum(pages_per_seq)
+    max_pp = max(pages_per_seq + [1]) if max_pages_per_seq is None else int(max_pages_per_seq)
+    poison = n_used
+    q = _randn_bf16(gen, (B, 1, Hq, D))
+    k_pool = _randn_bf16(gen, (n_used + 1, page_size, Hkv, D))
+    v_pool = _randn_bf16(gen, (n_used + 1, page_size, Hkv, D))
+
+    def sentinel(shape):
+        sign = torch.randint(0, 2, shape, generator=gen, dtype=torch.int16) * 2 - 1
+        return (sign.to(torch.float32) * SENTINEL).to(torch.bfloat16)
+
+    k_pool[poison] = sentinel(k_pool[poison].shape)
+    v_pool[poison] = sentinel(v_pool[poison].shape)
+    perm = torch.randperm(n_used, generator=gen).to(torch.int32)
+    table = torch.full((B, max_pp), poison, dtype=torch.int32)
+    cursor = 0
+    for b, npg in enumerate(pages_per_seq):
+        table[b, :npg] = perm[cursor:cursor + npg]
+        cursor += npg
+        L = int(seqlens[b])
+        if npg and L % page_size:
+            last = int(table[b, npg - 1])
+            k_pool[last, L % page_size:] = sentinel(k_pool[last, L % page_size:].shape)
+            v_pool[last, L % page_size:] = sentinel(v_pool[last, L % page_size:].shape)
+    return PagedKV(q, k_pool, v_pool, table, seqlens.clone(), page_size)
+
+
+def gqa_decode_config_inputs(cfg: GqaDecodeConfig = GQA_DECODE_CONFIG):
+    gen = torch.Generator(device="cpu").manual_seed(int(cfg.seed))
+    seqlens = torch.randint(cfg.min_len, cfg.max_len + 1, (cfg.B,), generator=gen, dtype=torch.int32)
+    return paged_gqa_decode_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, seqlens, cfg.page_size, cfg.seed + 100000)
 
 
 def decode_config_inputs(cfg: DecodeConfig = DECODE_CONFIG):

@@ -25,6 +25,10 @@ What it computes is the plain definition the fused kernels must reach exactly
   and V is its first 512 entries.
 * "FlashMLA" page, technical basis list: the KV cache is paged with 64-token
   pages; a block table maps each sequence's logical page to a physical page.
+* "GQLA: Group-Query Latent Attention ...", key terms (GQA path): each group
+  of query heads reads its own group-expanded cache.  Here that is a paged
+  cache of separate K and V rows per (token, KV head); query head h reads KV
+  head h // (Hq / Hkv), as in the dense oracle.
 
 Outputs: O (fp64) and LSE = ln sum_j exp(S_ij) (fp64, natural log of the sum
 over the *scaled* scores).  A row with no visible key has O = 0, LSE = -inf.
@@ -42,7 +46,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention", "decode_paged", "gather_pages"]
+__all__ = ["attention", "decode_paged", "decode_paged_gqa", "gather_pages"]
 
 
 def _rows_softmax_weighted(S: np.ndarray, V: np.ndarray):
@@ -151,4 +155,39 @@ def decode_paged(q, kv_pages, block_table, cache_seqlens, scale: float, dv: int,
         o, lse = _rows_softmax_weighted(S, Vmat)
         O[b] = o
         LSE[b] = lse
+    return O, LSE
+
+
+def decode_paged_gqa(q, k_pages, v_pages, block_table, cache_seqlens, scale: float, page_size: int = 64,
+                     seqs=None):
+    """GQA-path decode over a paged, group-expanded cache (one query token per sequence).
+
+    q: [B, Hq, D]; k_pages, v_pages: [num_pages, page_size, Hkv, D];
+    block_table: [B, max_pages] int; cache_seqlens: [B] int.  Query head h
+    attends, with no mask inside the sequence, to the K and V rows of KV head
+    h // (Hq // Hkv) of every cached token of its sequence.  seqs: optional
+    subset of sequences.  Returns O [len(seqs), Hq, D] and LSE [len(seqs), Hq]
+    in fp64; a sequence of length 0 gives O = 0 and LSE = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_pages = np.asarray(k_pages, dtype=np.float64)
+    v_pages = np.asarray(v_pages, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = k_pages.shape[2]
+    group = Hq // Hkv
+    bs = np.arange(B) if seqs is None else np.asarray(seqs, dtype=np.int64)
+    O = np.zeros((len(bs), Hq, D), dtype=np.float64)
+    LSE = np.full((len(bs), Hq), -np.inf, dtype=np.float64)
+    for i, b in enumerate(bs):
+        L = int(cache_seqlens[b])
+        if L == 0:
+            continue
+        for g in range(Hkv):
+            Kmat = gather_pages(k_pages[:, :, g, :], block_table[b], L, page_size)
+            Vmat = gather_pages(v_pages[:, :, g, :], block_table[b], L, page_size)
+            heads = np.arange(g * group, (g + 1) * group)
+            S = scale * (q[b, heads, :] @ Kmat.T)
+            o, lse = _rows_softmax_weighted(S, Vmat)
+            O[i, heads] = o
+            LSE[i, heads] = lse
     return O, LSE
