@@ -19,8 +19,8 @@ import re
 
 import torch
 
-__all__ = ["fwd", "decode_paged", "decode_paged_noalloc", "decode_workspace_size", "read_device_status",
-           "library", "AttnError", "exported_symbols", "STATUS"]
+__all__ = ["fwd", "decode_paged", "decode_paged_noalloc", "decode_workspace_size", "decode_paged_gqa",
+           "decode_gqa_workspace_size", "read_device_status", "library", "AttnError", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libattn_b200.so")
@@ -53,6 +53,8 @@ _SIGNATURES = {
     "attn_decode_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_decode_paged_noalloc_max_bytes": (_sz, []),
     "attn_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "attn_decode_paged_gqa_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
 }
 
 
@@ -205,6 +207,52 @@ def decode_paged_noalloc(q: torch.Tensor, kv_pages: torch.Tensor, block_table: t
                                                  Dk, dv, page_size, num_pages, block_table.shape[1], float(scale),
                                                  _stream_handle(q.device))
     _check(rc, "attn_decode_paged_noalloc")
+    return out, lse
+
+
+def decode_gqa_workspace_size(B: int, Hq: int, Hkv: int, D: int, device=None) -> int:
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D))
+
+
+def decode_paged_gqa(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                     cache_seqlens: torch.Tensor, scale: float, out: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """GQA-path paged decode, one query token per sequence.
+
+    q [B,1,Hq,D] bf16; k_pages, v_pages [num_pages,page_size,Hkv,D] bf16;
+    block_table [B,max_pages] int32; cache_seqlens [B] int32.
+    Returns (o [B,1,Hq,D] bf16, lse [B,Hq] fp32).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    B, sq, Hq, D = q.shape
+    num_pages, page_size, Hkv, D2 = k_pages.shape
+    if (sq != 1 or D2 != D or tuple(v_pages.shape) != tuple(k_pages.shape) or block_table.shape[0] != B
+            or cache_seqlens.shape[0] != B):
+        raise ValueError("decode_paged_gqa shape mismatch")
+    if out is None:
+        out = torch.empty((B, 1, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 2)
+    with torch.cuda.device(q.device):
+        need = int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D))
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
+            raise ValueError("workspace too small")
+        rc = library().attn_decode_paged_gqa(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                             block_table.data_ptr(), cache_seqlens.data_ptr(), out.data_ptr(),
+                                             lse.data_ptr(), B, Hq, Hkv, D, page_size, num_pages,
+                                             block_table.shape[1], float(scale), workspace.data_ptr(),
+                                             workspace.numel() * workspace.element_size(),
+                                             _stream_handle(q.device))
+    _check(rc, "attn_decode_paged_gqa")
     return out, lse
 
 

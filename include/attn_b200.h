@@ -150,6 +150,47 @@ int attn_decode_paged_noalloc(const void* q, const void* kv_pages, const int32_t
 size_t attn_decode_paged_noalloc_max_bytes(void);
 
 /*
+ * attn_decode_paged_gqa_workspace_size: bytes of device workspace that
+ * attn_decode_paged_gqa needs for B sequences, Hq query heads in groups of
+ * Hq / Hkv, head dim D, on the current device (0 for an unsupported shape).
+ */
+size_t attn_decode_paged_gqa_workspace_size(int B, int Hq, int Hkv, int D);
+
+/*
+ * attn_decode_paged_gqa: one new query token per sequence attending to a
+ * paged cache of separate K and V rows per (token, KV head): the GQA decoding
+ * path ("GQLA: Group-Query Latent Attention ...", key terms: each group of
+ * query heads reads its own group-expanded cache; "FlashMLA" page: 64-token
+ * pages reached through a block table).
+ *
+ *   q             [B, 1, Hq, D] bf16
+ *   k_pages       [num_pages, page_size, Hkv, D] bf16
+ *   v_pages       [num_pages, page_size, Hkv, D] bf16
+ *   block_table   [B, max_pages_per_seq] int32 (token t of sequence b lives in
+ *                 page block_table[b][t / page_size], row t % page_size)
+ *   cache_seqlens [B] int32
+ *   o             [B, 1, Hq, D] bf16 (written)
+ *   lse           [B, Hq] fp32 (written), natural-log LSE of the scaled scores
+ *   workspace     device scratch of at least
+ *                 attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D) bytes,
+ *                 256-byte aligned; contents irrelevant on entry.
+ *
+ * Query head h reads KV head h / (Hq / Hkv) and sees every cached token of its
+ * sequence.  A sequence of length 0 gets O = 0 and LSE = -inf.  Rows past the
+ * sequence length must hold finite values (they may be read).
+ *
+ * Supported: D in {64, 128}; Hq / Hkv in {1, 2, 4, 8}; page_size = 64;
+ * B <= 2048; pointers 16-byte aligned.  Block-table entries out of
+ * [0, num_pages) make the kernel read page 0 instead for that page and record
+ * ATTN_ERR_INVALID_ARG in the device status word.  Accumulation is fp32; O is
+ * rounded to bf16 once.  Deterministic run to run.
+ */
+int attn_decode_paged_gqa(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                          const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                          int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * attn_selftest_wait_timeout: exercise the bounded-wait failure path.  The
  * source pages describe no counterpart; this checks this library's own
  * failure detection.  One CTA waits on a barrier that nothing ever releases,

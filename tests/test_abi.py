@@ -72,3 +72,29 @@ def test_fwd_no_keys_accepts_null_kv_and_empty_query(lib):
 def test_selftest_rejects_bad_limits_on_host(lib):
     assert lib.attn_selftest_wait_timeout(0, None) == 1
     assert lib.attn_selftest_wait_timeout(20_000_000, None) == 1
+
+
+def _gqa(lib, q=A, kp=A, vp=A, bt=A, sl=A, o=A, lse=A, B=2, Hq=8, Hkv=2, D=128, page=64, npages=4, maxp=2,
+         scale=0.1, ws=A, ws_bytes=1 << 20):
+    return lib.attn_decode_paged_gqa(q, kp, vp, bt, sl, o, lse, B, Hq, Hkv, D, page, npages, maxp, scale, ws,
+                                     ws_bytes, None)
+
+
+def test_gqa_decode_rejects_bad_arguments(lib):
+    assert _gqa(lib, q=None) == 1
+    assert _gqa(lib, vp=None) == 1
+    assert _gqa(lib, kp=A + 8) == 1          # misaligned
+    assert _gqa(lib, sl=A + 2) == 1
+    assert _gqa(lib, Hq=6, Hkv=4) == 1       # Hq % Hkv
+    assert _gqa(lib, B=0) == 1
+    assert _gqa(lib, npages=0) == 1
+    assert _gqa(lib, scale=0.0) == 1
+    assert _gqa(lib, scale=float("nan")) == 1
+
+
+def test_gqa_decode_unsupported_shapes(lib):
+    assert _gqa(lib, D=96) == 2
+    assert _gqa(lib, D=256) == 2
+    assert _gqa(lib, Hq=32, Hkv=2) == 2      # group of 16
+    assert _gqa(lib, page=16) == 2
+    assert _gqa(lib, B=5000) == 2
