@@ -16,13 +16,14 @@
 //
 // Work split: the (sequence, KV head) units are laid end to end, each as its
 // ceil(L_b/64) pages, and the resulting page list is cut into one contiguous
-// equal range per worker.  A worker is one warp: it owns a two-stage ring of
-// (K page tile, V page tile) pairs for one KV head, issues its own TMA loads
-// (lane 0) two pages ahead of the page it computes, and walks its range
-// unit by unit.  A unit read entirely by one worker is written out directly;
-// the pieces of a unit split between workers are written as fp32 partials
-// (O normalised by its own sum, plus LSE) and merged by the LSE-combine
-// kernel.
+// equal range per worker.  A worker is one warp (four per SM, one per
+// scheduler): it owns a ring of page tiles for one KV head, loaded in the
+// order they are used (K of page k, V of page k, K of page k+1, ...) and each
+// released as soon as its product is done, issues its own TMA loads (lane 0)
+// and walks its range unit by unit.  A unit read entirely by one worker is
+// written out directly; the pieces of a unit split between workers are
+// written as fp32 partials (O normalised by its own sum, plus LSE) and merged
+// by the LSE-combine kernel.
 //
 // Per page (64 tokens) a worker computes, lane = token for the scores (two
 // tokens per lane) and lane = output dims for the product:
@@ -39,7 +40,6 @@ namespace gqa {
 
 constexpr int PAGE = 64;
 constexpr int B_MAX = 2048;
-constexpr int STAGES = 2;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -49,18 +49,20 @@ struct Cfg {
   static constexpr int G = G_;
   static constexpr int CHUNKS = D / 64;                   // 128-byte column chunks of a row
   static constexpr int CHUNK_BYTES = PAGE * 128;          // one TMA box: 64 tokens x 64 dims
-  static constexpr int KV_BYTES = CHUNKS * CHUNK_BYTES;   // K (or V) rows of one page, one KV head
-  static constexpr int STAGE_BYTES = 2 * KV_BYTES;        // K tile then V tile
+  static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES; // K (or V) rows of one page, one KV head
+  // Tiles per worker: with three, K of page k+1 and V of page k+1 load while
+  // the products of page k run (two tiles in flight per worker).
+  static constexpr int TILES = (D == 128) ? 3 : 6;
   static constexpr int Q_BYTES = G * D * 4;               // fp32, pre-scaled by scale*log2e
   static constexpr int P_BYTES = PAGE * G * 4;            // fp32 [token][head]
-  static constexpr int WORKER_BYTES = STAGES * STAGE_BYTES + Q_BYTES + P_BYTES;
+  static constexpr int WORKER_BYTES = TILES * TILE_BYTES + Q_BYTES + P_BYTES;
   static constexpr int WORKER_STRIDE = (WORKER_BYTES + 1023) / 1024 * 1024;
-  static constexpr int WORKERS = (D == 128) ? 3 : 5;      // as many as shared memory holds
+  static constexpr int WORKERS = 4;                       // one warp per scheduler of the SM
   static constexpr int THREADS = 32 * WORKERS;
   static constexpr int DPL = D / 32;                      // output dims per lane
   static constexpr int OFF_PREF = WORKERS * WORKER_STRIDE;
   static constexpr int OFF_BAR = (OFF_PREF + (B_MAX + 1) * 4 + 7) / 8 * 8;
-  static constexpr int OFF_MISC = OFF_BAR + WORKERS * STAGES * 8;
+  static constexpr int OFF_MISC = OFF_BAR + WORKERS * TILES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(D == 64 || D == 128, "head dim");
@@ -166,12 +168,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t wbase = base + warp * C::WORKER_STRIDE;
-  float* q_s = reinterpret_cast<float*>(base_ptr + warp * C::WORKER_STRIDE + STAGES * C::STAGE_BYTES);
+  constexpr int TILES = C::TILES;
+  float* q_s = reinterpret_cast<float*>(base_ptr + warp * C::WORKER_STRIDE + TILES * C::TILE_BYTES);
   float* p_s = q_s + G * D;
-  auto full_bar = [&](int st) -> uint32_t { return base + C::OFF_BAR + 8u * (warp * STAGES + st); };
+  auto full_bar = [&](int slot) -> uint32_t { return base + C::OFF_BAR + 8u * (warp * TILES + slot); };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::WORKERS * STAGES; ++i) mbar_init(base + C::OFF_BAR + 8u * i, 1);
+    for (int i = 0; i < C::WORKERS * TILES; ++i) mbar_init(base + C::OFF_BAR + 8u * i, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -211,45 +214,43 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int R0 = range_start(worker, T, a.workers), R1 = range_start(worker + 1, T, a.workers);
 
   // ---------------------------------------------------------------- loads
-  // A second cursor walks the same range and issues the TMA loads of the
-  // page that will be computed two pages later into the stage just freed.
+  // Tile n of this worker (n = 2 * page + 0 for K, + 1 for V, pages counted in
+  // range order) goes to slot n % TILES, phase n / TILES.  A second cursor
+  // walks the same range and issues the next tile whenever a slot frees up.
   UnitWalk lw;
   lw.init(pref, a.B, a.Hkv, R0, R1);
   int l_b = 0, l_g = 0, l_x = 0, l_x1 = 0, l_u0 = 0;
   bool l_more = lw.next(l_b, l_g, l_x, l_x1, l_u0);
-  int loads = 0;
+  int tiles = 0;   // tiles issued
   auto issue_next = [&]() {
     if (!l_more) return;
-    const int st = loads % STAGES;
+    const int slot = tiles % TILES;
+    const bool is_v = tiles & 1;
     if (lane == 0) {
       int page = a.block_table[(size_t)l_b * a.max_pages + (l_x - l_u0)];
       if (page < 0 || page >= a.num_pages) {
-        atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
+        if (!is_v) atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
         page = 0;   // never read outside the pool; the result of this sequence is undefined
       }
-      // the generic-proxy reads of this stage (previous page) happen before the async-proxy writes
+      // the generic-proxy reads of this slot (an earlier tile) happen before the async-proxy writes
       fence_proxy_async_smem();
-      const uint32_t bar = full_bar(st);
-      mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-      const uint32_t dst = wbase + st * C::STAGE_BYTES;
+      const uint32_t bar = full_bar(slot);
+      mbar_arrive_expect_tx(bar, C::TILE_BYTES);
+      const uint32_t dst = wbase + slot * C::TILE_BYTES;
 #pragma unroll
-      for (int c = 0; c < C::CHUNKS; ++c) {
-        tma_load_3d(dst + c * C::CHUNK_BYTES, &tm_k, bar, c * 64, l_g, page * PAGE);
-        tma_load_3d(dst + C::KV_BYTES + c * C::CHUNK_BYTES, &tm_v, bar, c * 64, l_g, page * PAGE);
-      }
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_3d(dst + c * C::CHUNK_BYTES, is_v ? &tm_v : &tm_k, bar, c * 64, l_g, page * PAGE);
     }
-    ++loads;
-    if (++l_x == l_x1) {
-      l_more = lw.next(l_b, l_g, l_x, l_x1, l_u0);
-    }
+    ++tiles;
+    if (is_v && ++l_x == l_x1) l_more = lw.next(l_b, l_g, l_x, l_x1, l_u0);
   };
-  for (int i = 0; i < STAGES; ++i) issue_next();
+  for (int i = 0; i < TILES; ++i) issue_next();
 
   // ---------------------------------------------------------------- compute
   UnitWalk w;
   w.init(pref, a.B, a.Hkv, R0, R1);
   int sb, sg, x0, x1, u0;
-  int k = 0;   // pages computed by this worker
+  int k = 0;   // pages computed by this worker (tiles 2k and 2k + 1)
   bool ok = true;
   const float sl2 = a.scale_log2;
   while (ok && w.next(sb, sg, x0, x1, u0)) {
@@ -265,27 +266,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     __syncwarp();
     float m_run[G], l_lane[G];
-    uint64_t o_acc[G][DPL / 2];
+    uint64_t o_acc[2][G][DPL / 2];   // two sets (even and odd tokens)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_run[h] = -INFINITY;
       l_lane[h] = 0.f;
 #pragma unroll
-      for (int j = 0; j < DPL / 2; ++j) o_acc[h][j] = f2_pack(0.f, 0.f);
+      for (int j = 0; j < DPL / 2; ++j) o_acc[0][h][j] = o_acc[1][h][j] = f2_pack(0.f, 0.f);
     }
     for (int x = x0; x < x1; ++x, ++k) {
-      const int st = k % STAGES;
-      if (!warp_wait(full_bar(st), (k / STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
-      const uint32_t kt = wbase + st * C::STAGE_BYTES;
-      const uint32_t vt = kt + C::KV_BYTES;
+      const int nk = 2 * k, nv = 2 * k + 1;
+      if (!warp_wait(full_bar(nk % TILES), (nk / TILES) & 1, abort_flag, a.status)) { ok = false; break; }
+      const uint32_t kt = wbase + (nk % TILES) * C::TILE_BYTES;
+      const uint32_t vt = wbase + (nv % TILES) * C::TILE_BYTES;
       const int valid = L - (x - u0) * PAGE;   // tokens of this page inside the sequence (>= 1)
 
       // ---- scores: lane = tokens lane and lane + 32
-      uint64_t acc[2][G];
+      // two accumulator sets (even and odd 8-dim chunks) double the
+      // independent FMA chains
+      uint64_t acc[2][2][G];
 #pragma unroll
-      for (int tt = 0; tt < 2; ++tt)
+      for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[tt][h] = f2_pack(0.f, 0.f);
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+          for (int h = 0; h < G; ++h) acc[e][tt][h] = f2_pack(0.f, 0.f);
 #pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
         const int cc = c >> 3, jj = c & 7;
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[tt][h] = f2_fma(kp[j], qv[h][j], acc[tt][h]);
+            for (int j = 0; j < 4; ++j) acc[c & 1][tt][h] = f2_fma(kp[j], qv[h][j], acc[c & 1][tt][h]);
         }
       }
       float s[2][G];
@@ -322,10 +327,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float lo, hi;
-          f2_unpack(acc[tt][h], lo, hi);
+          f2_unpack(f2_add(acc[0][tt][h], acc[1][tt][h]), lo, hi);
           s[tt][h] = live ? lo + hi : -INFINITY;
         }
       }
+
+      __syncwarp();   // every lane is done with the K tile
+      issue_next();   // refill its slot
 
       // ---- online softmax (m, the rescale decision and alpha are warp-uniform)
       float pr[2][G];
@@ -344,7 +352,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const float alpha = ex2(m_run[h] - m_use);
           l_lane[h] *= alpha;
 #pragma unroll
-          for (int j = 0; j < DPL / 2; ++j) o_acc[h][j] = f2_mul(o_acc[h][j], f2_pack(alpha, alpha));
+          for (int j = 0; j < DPL / 2; ++j) {
+            o_acc[0][h][j] = f2_mul(o_acc[0][h][j], f2_pack(alpha, alpha));
+            o_acc[1][h][j] = f2_mul(o_acc[1][h][j], f2_pack(alpha, alpha));
+          }
         }
         l_lane[h] += pr[0][h] + pr[1][h];
         m_run[h] = m_use;
@@ -365,6 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       __syncwarp();
 
       // ---- O += P V: lane = output dims [DPL*lane, DPL*lane + DPL)
+      if (!warp_wait(full_bar(nv % TILES), (nv / TILES) & 1, abort_flag, a.status)) { ok = false; break; }
       const int dim0 = DPL * lane;
       const int cc = dim0 >> 6;                 // column chunk
       const int byte_in_row = (dim0 & 63) * 2;  // within the 128-byte row
@@ -404,10 +416,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int h = 0; h < G; ++h)
 #pragma unroll
-          for (int j = 0; j < DPL / 2; ++j) o_acc[h][j] = f2_fma(vp[j], f2_pack(pv[h], pv[h]), o_acc[h][j]);
+          for (int j = 0; j < DPL / 2; ++j)
+            o_acc[t & 1][h][j] = f2_fma(vp[j], f2_pack(pv[h], pv[h]), o_acc[t & 1][h][j]);
       }
-      __syncwarp();   // every lane is done with this stage and with p_s
-      issue_next();   // refill the stage just read
+      __syncwarp();   // every lane is done with the V tile and with p_s
+      issue_next();   // refill its slot
     }
     if (!ok) break;
 
@@ -424,7 +437,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       float ov[DPL];
 #pragma unroll
       for (int j = 0; j < DPL / 2; ++j) {
-        f2_unpack(o_acc[h][j], ov[2 * j], ov[2 * j + 1]);
+        f2_unpack(f2_add(o_acc[0][h][j], o_acc[1][h][j]), ov[2 * j], ov[2 * j + 1]);
         ov[2 * j] *= inv_l;
         ov[2 * j + 1] *= inv_l;
       }
@@ -453,7 +466,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   // Drain: every issued load must land before the CTA's shared memory goes away.
   if (lane == 0)
-    for (int j = max(k, loads - STAGES); j < loads; ++j) mbar_wait_drain(full_bar(j % STAGES), (j / STAGES) & 1);
+    for (int n = max(0, tiles - TILES); n < tiles; ++n) mbar_wait_drain(full_bar(n % TILES), (n / TILES) & 1);
   __syncwarp();
 }
 
