@@ -16,17 +16,20 @@
 //
 // Work split: the (sequence, KV head) units are laid end to end, each as its
 // ceil(L_b/64) pages, and the resulting page list is cut into one contiguous
-// equal range per worker.  A worker is one warp (four per SM, one per
-// scheduler): it owns a ring of page tiles for one KV head, loaded in the
-// order they are used (K of page k, V of page k, K of page k+1, ...) and each
-// released as soon as its product is done, issues its own TMA loads (lane 0)
-// and walks its range unit by unit.  A unit read entirely by one worker is
+// equal range per worker.  A worker is a pair of warps (four pairs per SM,
+// two warps per scheduler): it owns a ring of page tiles for one KV head,
+// loaded in the order they are used (K of page k, V of page k, K of page
+// k+1, ...) and each released as soon as both warps are done with it; the
+// first warp issues the TMA loads (lane 0).  Each warp takes 32 of the 64
+// tokens of every page for both products; the pair agrees on the row max of
+// the page through shared memory and merges its sums and O at the end of a
+// unit.  A unit read entirely by one worker is
 // written out directly; the pieces of a unit split between workers are
 // written as fp32 partials (O normalised by its own sum, plus LSE) and merged
 // by the LSE-combine kernel.
 //
-// Per page (64 tokens) a worker computes, lane = token for the scores (two
-// tokens per lane) and lane = output dims for the product:
+// Per page (64 tokens) a warp computes, lane = token for the scores (one of
+// its 32 tokens per lane) and lane = output dims for the product:
 //   s[t][h] = q[h] . k[t]   (q pre-scaled by scale*log2e, fp32 in smem)
 //   warp max per head, lazy rescale (only when the max grew by > 2^8),
 //   p[t][h] = 2^(s - m) -> smem, O[h][dims of this lane] += sum_t p[t][h] v[t]
@@ -55,12 +58,15 @@ struct Cfg {
   static constexpr int TILES = (D == 128) ? 3 : 6;
   static constexpr int Q_BYTES = G * D * 4;               // fp32, pre-scaled by scale*log2e
   static constexpr int P_BYTES = PAGE * G * 4;            // fp32 [token][head]
-  static constexpr int WORKER_BYTES = TILES * TILE_BYTES + Q_BYTES + P_BYTES;
-  static constexpr int WORKER_STRIDE = (WORKER_BYTES + 1023) / 1024 * 1024;
-  static constexpr int WORKERS = 4;                       // one warp per scheduler of the SM
-  static constexpr int THREADS = 32 * WORKERS;
+  static constexpr int X_BYTES = 2 * G * 4;               // row max / sum exchange of a warp pair
+  static constexpr int QPX_BYTES = (Q_BYTES + P_BYTES + X_BYTES + 15) / 16 * 16;
+  // A worker is a pair of warps sharing one tile ring: four workers fill an
+  // SM with two warps per scheduler.
+  static constexpr int WORKERS = 4;
+  static constexpr int THREADS = 64 * WORKERS;
   static constexpr int DPL = D / 32;                      // output dims per lane
-  static constexpr int OFF_PREF = WORKERS * WORKER_STRIDE;
+  static constexpr int OFF_QPX = WORKERS * TILES * TILE_BYTES;   // tile rings first (1024-aligned)
+  static constexpr int OFF_PREF = OFF_QPX + WORKERS * QPX_BYTES;
   static constexpr int OFF_BAR = (OFF_PREF + (B_MAX + 1) * 4 + 7) / 8 * 8;
   static constexpr int OFF_MISC = OFF_BAR + WORKERS * TILES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -158,7 +164,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const Args a) {
-  constexpr int D = C::D, G = C::G, DPL = C::DPL;
+  constexpr int D = C::D, G = C::G, DPL = C::DPL, TILES = C::TILES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -167,11 +173,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::OFF_MISC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t wbase = base + warp * C::WORKER_STRIDE;
-  constexpr int TILES = C::TILES;
-  float* q_s = reinterpret_cast<float*>(base_ptr + warp * C::WORKER_STRIDE + TILES * C::TILE_BYTES);
-  float* p_s = q_s + G * D;
-  auto full_bar = [&](int slot) -> uint32_t { return base + C::OFF_BAR + 8u * (warp * TILES + slot); };
+  const int pw = warp >> 1;     // worker = pair of warps
+  const int half = warp & 1;    // this warp's tokens of every page: [32 half, 32 half + 32)
+  const uint32_t wbase = base + pw * TILES * C::TILE_BYTES;
+  float* q_s = reinterpret_cast<float*>(base_ptr + C::OFF_QPX + pw * C::QPX_BYTES);   // [G][D]
+  float* p_s = q_s + G * D;                                                              // [64][G]
+  float* x_s = p_s + PAGE * G;                                                           // [2][G]
+  auto full_bar = [&](int slot) -> uint32_t { return base + C::OFF_BAR + 8u * (pw * TILES + slot); };
+  const int pair_bar = 1 + pw;
+  auto pair_sync = [&]() { named_bar_sync(pair_bar, 64); };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::WORKERS * TILES; ++i) mbar_init(base + C::OFF_BAR + 8u * i, 1);
@@ -210,20 +220,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int T = a.Hkv * pref[a.B];
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i <= a.B; i += C::THREADS) a.ws_pref[i] = pref[i];
-  const int worker = blockIdx.x * C::WORKERS + warp;
+  const int worker = blockIdx.x * C::WORKERS + pw;
   const int R0 = range_start(worker, T, a.workers), R1 = range_start(worker + 1, T, a.workers);
+  bool ok = true;
 
   // ---------------------------------------------------------------- loads
   // Tile n of this worker (n = 2 * page + 0 for K, + 1 for V, pages counted in
-  // range order) goes to slot n % TILES, phase n / TILES.  A second cursor
-  // walks the same range and issues the next tile whenever a slot frees up.
+  // range order) goes to slot n % TILES, phase n / TILES.  The first warp of
+  // the pair walks the range a second time and issues the next tile whenever
+  // both warps have released a slot.
   UnitWalk lw;
   lw.init(pref, a.B, a.Hkv, R0, R1);
   int l_b = 0, l_g = 0, l_x = 0, l_x1 = 0, l_u0 = 0;
   bool l_more = lw.next(l_b, l_g, l_x, l_x1, l_u0);
-  int tiles = 0;   // tiles issued
+  int tiles = 0;   // tiles issued (meaningful in the first warp)
   auto issue_next = [&]() {
-    if (!l_more) return;
+    if (half != 0 || !l_more || !ok) return;
     const int slot = tiles % TILES;
     const bool is_v = tiles & 1;
     if (lane == 0) {
@@ -247,24 +259,27 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   for (int i = 0; i < TILES; ++i) issue_next();
 
   // ---------------------------------------------------------------- compute
+  // Both warps of the pair run the same walk and pass the same named barriers
+  // in the same order.  After a failed wait a warp keeps walking without
+  // touching shared tiles, so the barrier counts stay matched.
   UnitWalk w;
   w.init(pref, a.B, a.Hkv, R0, R1);
   int sb, sg, x0, x1, u0;
-  int k = 0;   // pages computed by this worker (tiles 2k and 2k + 1)
-  bool ok = true;
+  int k = 0;   // pages computed (tiles 2k and 2k + 1)
   const float sl2 = a.scale_log2;
-  while (ok && w.next(sb, sg, x0, x1, u0)) {
+  const int t_mine = 32 * half + lane;   // this lane's token of every page (scores)
+  while (w.next(sb, sg, x0, x1, u0)) {
     const int L = seq_len_eff(a.seqlens[sb], a.max_pages);
     const int np = pref[sb + 1] - pref[sb];
-    // q of the group's G heads, fp32, pre-scaled (the previous unit's reads of q_s are done)
-    __syncwarp();
-    for (int i = lane; i < G * D / 2; i += 32) {
+    // q of the group's G heads, fp32, pre-scaled; both warps load half of it
+    pair_sync();   // the previous unit's reads of q_s and x_s are done
+    for (int i = half * 32 + lane; i < G * D / 2; i += 64) {
       const uint32_t wq =
           reinterpret_cast<const uint32_t*>(a.q + ((size_t)sb * (a.Hkv * G) + sg * G) * D)[i];
       q_s[2 * i] = __uint_as_float(wq << 16) * sl2;
       q_s[2 * i + 1] = __uint_as_float(wq & 0xffff0000u) * sl2;
     }
-    __syncwarp();
+    pair_sync();
     float m_run[G], l_lane[G];
     uint64_t o_acc[2][G][DPL / 2];   // two sets (even and odd tokens)
 #pragma unroll
@@ -276,37 +291,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     for (int x = x0; x < x1; ++x, ++k) {
       const int nk = 2 * k, nv = 2 * k + 1;
-      if (!warp_wait(full_bar(nk % TILES), (nk / TILES) & 1, abort_flag, a.status)) { ok = false; break; }
       const uint32_t kt = wbase + (nk % TILES) * C::TILE_BYTES;
       const uint32_t vt = wbase + (nv % TILES) * C::TILE_BYTES;
       const int valid = L - (x - u0) * PAGE;   // tokens of this page inside the sequence (>= 1)
+      if (ok) ok = warp_wait(full_bar(nk % TILES), (nk / TILES) & 1, abort_flag, a.status);
 
-      // ---- scores: lane = tokens lane and lane + 32
-      // two accumulator sets (even and odd 8-dim chunks) double the
-      // independent FMA chains
-      uint64_t acc[2][2][G];
+      // ---- scores of this lane's token against the G heads
+      float s[G];
+      if (ok) {
+        uint64_t acc[2][G];
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
+        for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[e][tt][h] = f2_pack(0.f, 0.f);
+          for (int h = 0; h < G; ++h) acc[e][h] = f2_pack(0.f, 0.f);
+        const int t = t_mine;
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const int cc = c >> 3, jj = c & 7;
-        uint64_t qv[G][4];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float4 q0 = *reinterpret_cast<const float4*>(q_s + h * D + c * 8);
-          const float4 q1 = *reinterpret_cast<const float4*>(q_s + h * D + c * 8 + 4);
-          qv[h][0] = f2_pack(q0.x, q0.y);
-          qv[h][1] = f2_pack(q0.z, q0.w);
-          qv[h][2] = f2_pack(q1.x, q1.y);
-          qv[h][3] = f2_pack(q1.z, q1.w);
-        }
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int t = lane + 32 * tt;
+        for (int c = 0; c < D / 8; ++c) {
+          const int cc = c >> 3, jj = c & 7;
           uint32_t k0, k1, k2, k3;
           ld_shared_v4(kt + cc * C::CHUNK_BYTES + t * 128 + ((jj ^ (t & 7)) << 4), k0, k1, k2, k3);
           uint64_t kp[4];
@@ -315,157 +316,185 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           bf16x2_to_f2(k2, kp[2]);
           bf16x2_to_f2(k3, kp[3]);
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[c & 1][tt][h] = f2_fma(kp[j], qv[h][j], acc[c & 1][tt][h]);
+          for (int h = 0; h < G; ++h) {
+            const float4 q0 = *reinterpret_cast<const float4*>(q_s + h * D + c * 8);
+            const float4 q1 = *reinterpret_cast<const float4*>(q_s + h * D + c * 8 + 4);
+            acc[c & 1][h] = f2_fma(kp[0], f2_pack(q0.x, q0.y), acc[c & 1][h]);
+            acc[c & 1][h] = f2_fma(kp[1], f2_pack(q0.z, q0.w), acc[c & 1][h]);
+            acc[c & 1][h] = f2_fma(kp[2], f2_pack(q1.x, q1.y), acc[c & 1][h]);
+            acc[c & 1][h] = f2_fma(kp[3], f2_pack(q1.z, q1.w), acc[c & 1][h]);
+          }
         }
-      }
-      float s[2][G];
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        const bool live = lane + 32 * tt < valid;
+        const bool live = t < valid;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float lo, hi;
-          f2_unpack(f2_add(acc[0][tt][h], acc[1][tt][h]), lo, hi);
-          s[tt][h] = live ? lo + hi : -INFINITY;
+          f2_unpack(f2_add(acc[0][h], acc[1][h]), lo, hi);
+          s[h] = live ? lo + hi : -INFINITY;
+        }
+        // this warp's max per head
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float mx = s[h];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0) x_s[half * G + h] = mx;
         }
       }
+      pair_sync();    // both warps are done with the K tile and have posted their maxima
+      issue_next();   // refill the K tile's slot
 
-      __syncwarp();   // every lane is done with the K tile
-      issue_next();   // refill its slot
-
-      // ---- online softmax (m, the rescale decision and alpha are warp-uniform)
-      float pr[2][G];
+      // ---- online softmax over the page (m, the rescale decision and alpha
+      // are identical in both warps: the same two maxima, the same order)
+      if (ok) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float mx = fmaxf(s[0][h], s[1][h]);
+        for (int h = 0; h < G; ++h) {
+          const float mx = fmaxf(x_s[h], x_s[G + h]);
+          const float m_new = fmaxf(m_run[h], mx);
+          const bool grow = m_new > m_run[h] + kRescaleThreshold;
+          const float m_use = grow ? m_new : m_run[h];
+          const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
+          const float p = ex2(s[h] - m_eff);
+          if (grow) {
+            const float alpha = ex2(m_run[h] - m_use);
+            l_lane[h] *= alpha;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_new = fmaxf(m_run[h], mx);
-        const bool grow = m_new > m_run[h] + kRescaleThreshold;
-        const float m_use = grow ? m_new : m_run[h];
-        const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-        pr[0][h] = ex2(s[0][h] - m_eff);
-        pr[1][h] = ex2(s[1][h] - m_eff);
-        if (grow) {
-          const float alpha = ex2(m_run[h] - m_use);
-          l_lane[h] *= alpha;
-#pragma unroll
-          for (int j = 0; j < DPL / 2; ++j) {
-            o_acc[0][h][j] = f2_mul(o_acc[0][h][j], f2_pack(alpha, alpha));
-            o_acc[1][h][j] = f2_mul(o_acc[1][h][j], f2_pack(alpha, alpha));
+            for (int j = 0; j < DPL / 2; ++j) {
+              o_acc[0][h][j] = f2_mul(o_acc[0][h][j], f2_pack(alpha, alpha));
+              o_acc[1][h][j] = f2_mul(o_acc[1][h][j], f2_pack(alpha, alpha));
+            }
           }
+          l_lane[h] += p;
+          m_run[h] = m_use;
+          s[h] = p;
         }
-        l_lane[h] += pr[0][h] + pr[1][h];
-        m_run[h] = m_use;
-      }
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        float* dst = p_s + (lane + 32 * tt) * G;
+        float* dst = p_s + t_mine * G;
         if constexpr (G >= 4) {
 #pragma unroll
-          for (int h = 0; h < G; h += 4)
-            *reinterpret_cast<float4*>(dst + h) = make_float4(pr[tt][h], pr[tt][h + 1], pr[tt][h + 2], pr[tt][h + 3]);
+          for (int h = 0; h < G; h += 4) *reinterpret_cast<float4*>(dst + h) = make_float4(s[h], s[h + 1], s[h + 2], s[h + 3]);
         } else if constexpr (G == 2) {
-          *reinterpret_cast<float2*>(dst) = make_float2(pr[tt][0], pr[tt][1]);
+          *reinterpret_cast<float2*>(dst) = make_float2(s[0], s[1]);
         } else {
-          dst[0] = pr[tt][0];
+          dst[0] = s[0];
         }
+        __syncwarp();
+        ok = warp_wait(full_bar(nv % TILES), (nv / TILES) & 1, abort_flag, a.status);
       }
-      __syncwarp();
 
-      // ---- O += P V: lane = output dims [DPL*lane, DPL*lane + DPL)
-      if (!warp_wait(full_bar(nv % TILES), (nv / TILES) & 1, abort_flag, a.status)) { ok = false; break; }
-      const int dim0 = DPL * lane;
-      const int cc = dim0 >> 6;                 // column chunk
-      const int byte_in_row = (dim0 & 63) * 2;  // within the 128-byte row
-      const int unit = byte_in_row >> 4, in_unit = byte_in_row & 15;
+      // ---- O += P V over this warp's 32 tokens, lane = output dims
+      if (ok) {
+        const int dim0 = DPL * lane;
+        const int cc = dim0 >> 6;                 // column chunk
+        const int byte_in_row = (dim0 & 63) * 2;  // within the 128-byte row
+        const int unit = byte_in_row >> 4, in_unit = byte_in_row & 15;
 #pragma unroll 4
-      for (int t = 0; t < PAGE; ++t) {
-        const uint32_t addr = vt + cc * C::CHUNK_BYTES + t * 128 + ((unit ^ (t & 7)) << 4) + in_unit;
-        uint64_t vp[DPL / 2];
-        if constexpr (DPL == 4) {
-          uint32_t v0, v1;
-          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(addr));
-          bf16x2_to_f2(v0, vp[0]);
-          bf16x2_to_f2(v1, vp[1]);
-        } else {
-          uint32_t v0;
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v0) : "r"(addr));
-          bf16x2_to_f2(v0, vp[0]);
-        }
-        float pv[G];
-        const float* src = p_s + t * G;
-        if constexpr (G >= 4) {
-#pragma unroll
-          for (int h = 0; h < G; h += 4) {
-            const float4 f = *reinterpret_cast<const float4*>(src + h);
-            pv[h] = f.x;
-            pv[h + 1] = f.y;
-            pv[h + 2] = f.z;
-            pv[h + 3] = f.w;
+        for (int tt = 0; tt < 32; ++tt) {
+          const int t = 32 * half + tt;
+          const uint32_t addr = vt + cc * C::CHUNK_BYTES + t * 128 + ((unit ^ (t & 7)) << 4) + in_unit;
+          uint64_t vp[DPL / 2];
+          if constexpr (DPL == 4) {
+            uint32_t v0, v1;
+            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(addr));
+            bf16x2_to_f2(v0, vp[0]);
+            bf16x2_to_f2(v1, vp[1]);
+          } else {
+            uint32_t v0;
+            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v0) : "r"(addr));
+            bf16x2_to_f2(v0, vp[0]);
           }
-        } else if constexpr (G == 2) {
-          const float2 f = *reinterpret_cast<const float2*>(src);
-          pv[0] = f.x;
-          pv[1] = f.y;
-        } else {
-          pv[0] = src[0];
+          float pv[G];
+          const float* src = p_s + t * G;
+          if constexpr (G >= 4) {
+#pragma unroll
+            for (int h = 0; h < G; h += 4) {
+              const float4 f = *reinterpret_cast<const float4*>(src + h);
+              pv[h] = f.x;
+              pv[h + 1] = f.y;
+              pv[h + 2] = f.z;
+              pv[h + 3] = f.w;
+            }
+          } else if constexpr (G == 2) {
+            const float2 f = *reinterpret_cast<const float2*>(src);
+            pv[0] = f.x;
+            pv[1] = f.y;
+          } else {
+            pv[0] = src[0];
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int j = 0; j < DPL / 2; ++j)
+              o_acc[tt & 1][h][j] = f2_fma(vp[j], f2_pack(pv[h], pv[h]), o_acc[tt & 1][h][j]);
         }
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int j = 0; j < DPL / 2; ++j)
-            o_acc[t & 1][h][j] = f2_fma(vp[j], f2_pack(pv[h], pv[h]), o_acc[t & 1][h][j]);
       }
-      __syncwarp();   // every lane is done with the V tile and with p_s
-      issue_next();   // refill its slot
+      pair_sync();    // both warps are done with the V tile (and with this page's maxima)
+      issue_next();   // refill the V tile's slot
     }
-    if (!ok) break;
 
-    // ---- unit piece done: reduce the sum, write O (final or partial) and LSE
-    const bool complete = (x0 == u0) && (x1 == u0 + np);
-    const int slot = 2 * worker + (x0 == R0 ? 0 : 1);
+    // ---- unit piece done: the second warp hands its sums and O to the first
+    float l_w[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float l = l_lane[h];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const float lse = (l > 0.f) ? (m_run[h] + log2f(l)) * kLn2 : -INFINITY;
-      float ov[DPL];
+      l_w[h] = l;
+    }
+    if (half == 1 && ok) {
 #pragma unroll
-      for (int j = 0; j < DPL / 2; ++j) {
-        f2_unpack(f2_add(o_acc[0][h][j], o_acc[1][h][j]), ov[2 * j], ov[2 * j + 1]);
-        ov[2 * j] *= inv_l;
-        ov[2 * j + 1] *= inv_l;
+      for (int h = 0; h < G; ++h) {
+        if (lane == 0) x_s[h] = l_w[h];
+#pragma unroll
+        for (int j = 0; j < DPL / 2; ++j) {
+          float lo, hi;
+          f2_unpack(f2_add(o_acc[0][h][j], o_acc[1][h][j]), lo, hi);
+          q_s[h * D + DPL * lane + 2 * j] = lo;       // q is no longer needed for this unit
+          q_s[h * D + DPL * lane + 2 * j + 1] = hi;
+        }
       }
-      const int head = sg * G + h;
-      if (complete) {
-        __nv_bfloat16* dst = a.o + ((size_t)sb * (a.Hkv * G) + head) * D + DPL * lane;
-        if constexpr (DPL == 4) {
-          uint2 u;
-          u.x = pack_bf16x2(ov[0], ov[1]);
-          u.y = pack_bf16x2(ov[2], ov[3]);
-          *reinterpret_cast<uint2*>(dst) = u;
-        } else {
-          *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(ov[0], ov[1]);
+    }
+    pair_sync();
+    if (half == 0 && ok && !*abort_flag) {
+      const bool complete = (x0 == u0) && (x1 == u0 + np);
+      const int slot = 2 * worker + (x0 == R0 ? 0 : 1);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float l = l_w[h] + x_s[h];
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float lse = (l > 0.f) ? (m_run[h] + log2f(l)) * kLn2 : -INFINITY;
+        float ov[DPL];
+#pragma unroll
+        for (int j = 0; j < DPL / 2; ++j) {
+          f2_unpack(f2_add(o_acc[0][h][j], o_acc[1][h][j]), ov[2 * j], ov[2 * j + 1]);
+          ov[2 * j] = (ov[2 * j] + q_s[h * D + DPL * lane + 2 * j]) * inv_l;
+          ov[2 * j + 1] = (ov[2 * j + 1] + q_s[h * D + DPL * lane + 2 * j + 1]) * inv_l;
         }
-        if (lane == 0) a.lse[(size_t)sb * (a.Hkv * G) + head] = lse;
-      } else {
-        float* dst = a.ws_o + ((size_t)slot * G + h) * D + DPL * lane;
-        if constexpr (DPL == 4) {
-          *reinterpret_cast<float4*>(dst) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+        const int head = sg * G + h;
+        if (complete) {
+          __nv_bfloat16* dst = a.o + ((size_t)sb * (a.Hkv * G) + head) * D + DPL * lane;
+          if constexpr (DPL == 4) {
+            uint2 u;
+            u.x = pack_bf16x2(ov[0], ov[1]);
+            u.y = pack_bf16x2(ov[2], ov[3]);
+            *reinterpret_cast<uint2*>(dst) = u;
+          } else {
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(ov[0], ov[1]);
+          }
+          if (lane == 0) a.lse[(size_t)sb * (a.Hkv * G) + head] = lse;
         } else {
-          *reinterpret_cast<float2*>(dst) = make_float2(ov[0], ov[1]);
+          float* dst = a.ws_o + ((size_t)slot * G + h) * D + DPL * lane;
+          if constexpr (DPL == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+          } else {
+            *reinterpret_cast<float2*>(dst) = make_float2(ov[0], ov[1]);
+          }
+          if (lane == 0) a.ws_lse[(size_t)slot * G + h] = lse;
         }
-        if (lane == 0) a.ws_lse[(size_t)slot * G + h] = lse;
       }
     }
   }
   // Drain: every issued load must land before the CTA's shared memory goes away.
-  if (lane == 0)
+  if (half == 0 && lane == 0)
     for (int n = max(0, tiles - TILES); n < tiles; ++n) mbar_wait_drain(full_bar(n % TILES), (n / TILES) & 1);
   __syncwarp();
 }
