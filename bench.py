@@ -8,11 +8,15 @@ already resident in device memory:
     (B=1, Hq=32, Hkv=8, N=16384, D=128, bf16, scale 1/sqrt(128));
   * decode:  attn_decode_paged on the MLA absorbed paged-decode workload
     (64 sequences x 128 heads, latent 576/512, 64-token pages, lengths
-    uniform on [1024, 8192]).
+    uniform on [1024, 8192]);
+  * gqa:     attn_decode_paged_gqa on the GQA-path paged-decode workload
+    (64 sequences x 32 query heads in 8 groups, D=128, separate K/V pages,
+    the same length mix).
 The headline metric is prefill TFLOP/s (4*Nq*Nk*D per head, halved for
-causal); the decode KV-cache GB/s (bytes of the latent rows of valid tokens
-over the time of the split + combine kernels) is reported in the "decode"
-object of the same line.  Both are compared with the measured B200 peaks.
+causal); the decode KV-cache GB/s (bytes of the K/V rows of valid tokens
+over the time of the decode + combine kernels) is reported in the "decode"
+and "gqa_decode" objects of the same line.  All are compared with the
+measured B200 peaks.
 
 With N > 1 (torchrun, one process per GPU) every rank runs the same
 independent workload (weak scaling, no collective on the data path); the
@@ -48,6 +52,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_BYTES = {
     "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
     "decode": 349399808 + 16235008,     # decode_split_kernel, MLA decode workload
+    "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.
@@ -200,6 +205,33 @@ def decode_part(ea, dev):
     return p
 
 
+def gqa_part(ea, dev):
+    cfg = inputs.GQA_DECODE_CONFIG
+    c = inputs.gqa_decode_config_inputs(cfg)
+    host = {"q": c.q.pin_memory(), "kp": c.k_pages.pin_memory(), "vp": c.v_pages.pin_memory(),
+            "bt": c.block_table.pin_memory(), "sl": c.cache_seqlens.pin_memory()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    d["o"] = torch.empty((cfg.B, 1, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=dev)
+    d["lse"] = torch.empty((cfg.B, cfg.Hq), dtype=torch.float32, device=dev)
+    d["ws"] = torch.empty(ea.decode_gqa_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, dev), dtype=torch.uint8,
+                          device=dev)
+    host["o"] = torch.empty(d["o"].shape, dtype=torch.bfloat16).pin_memory()
+    host["lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
+
+    def run():
+        ea.decode_paged_gqa(d["q"], d["kp"], d["vp"], d["bt"], d["sl"], cfg.scale, out=d["o"], lse=d["lse"],
+                            workspace=d["ws"])
+
+    p = Part("gqa", run, [(d[n], host[n]) for n in ("q", "kp", "vp", "bt", "sl")],
+             [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=2)
+    p.cfg = cfg
+    p.kv_bytes = c.kv_valid_bytes()
+    p.tokens = int(c.cache_seqlens.to(torch.int64).sum())
+    p.flops = 4.0 * cfg.Hq * cfg.D * p.tokens
+    p.ws_bytes = d["ws"].numel()
+    return p
+
+
 def time_parts(parts, steps, stream):
     """Times `steps` steps; each step runs every part once.  Returns total ms
     and per-part lists of per-launch ms (CUDA events on the launching stream)."""
@@ -256,6 +288,8 @@ def run_gpu(args):
         parts.append(prefill_part(ea, dev))
     if args.part in ("all", "decode"):
         parts.append(decode_part(ea, dev))
+    if args.part in ("all", "gqa"):
+        parts.append(gqa_part(ea, dev))
 
     for _ in range(args.warmup):
         for p in parts:
@@ -315,6 +349,25 @@ def run_gpu(args):
                     "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
             "workspace_bytes": p.ws_bytes,
         }
+    gqa_obj = None
+    if "gqa" in by:
+        p = by["gqa"]
+        gbs = p.kv_bytes / (launch_ms["gqa"] * 1e-3) / 1e9
+        gqa_obj = {
+            "metric": "KV-cache GB/s (GQA-path paged decode)",
+            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["gqa"]) / 1e9, 1), "unit": "GB/s",
+            "ms_per_launch": round(launch_ms["gqa"], 4),
+            "config": {"workload": p.cfg.name, "B": p.cfg.B, "Hq": p.cfg.Hq, "Hkv": p.cfg.Hkv, "D": p.cfg.D,
+                       "page_size": p.cfg.page_size, "lengths": f"uniform [{p.cfg.min_len}, {p.cfg.max_len}]",
+                       "tokens": p.tokens, "kv_bytes": p.kv_bytes, "scale": p.cfg.scale,
+                       "l2": "K/V cache 1.35 GB per step, larger than L2, no flush"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
+                         "traffic": NCU_TRAFFIC_BYTES["gqa"], "kernel": "gqa_decode_kernel + gqa_combine_kernel"},
+            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["gqa"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+            "workspace_bytes": p.ws_bytes,
+        }
     if "prefill" in by:
         p = by["prefill"]
         achieved = p.work / (launch_ms["prefill"] * 1e-3) / 1e12
@@ -340,9 +393,14 @@ def run_gpu(args):
         })
         if decode_obj:
             line["decode"] = decode_obj
+        if gqa_obj:
+            line["gqa_decode"] = gqa_obj
     else:
-        line.update({k: decode_obj[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
+        head = decode_obj if decode_obj else gqa_obj
+        line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
         line["config"]["step"] = step_parts
+        if decode_obj and gqa_obj:
+            line["gqa_decode"] = gqa_obj
     if rank == 0 and world == 1 and not args.no_cpu_baseline and "prefill" in by:
         line["cpu_baseline"] = cpu_baseline(args.baseline_rows)
     if world > 1:
@@ -441,7 +499,7 @@ def main():
     ap.add_argument("--baseline-rows", type=int, default=768,
                     help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa"], default="all",
                     help="time only one piece of the step (for profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()
