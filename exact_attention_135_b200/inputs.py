@@ -137,10 +137,11 @@ class PagedCache:
         return int(self.cache_seqlens.to(torch.int64).sum()) * dk * 2
 
 
-def paged_decode_inputs(B, Hq, Dk, seqlens, page_size, seed, max_pages_per_seq=None):
+def paged_decode_inputs(B, Hq, Dk, seqlens, page_size, seed, max_pages_per_seq=None, s_q=1):
     """Build a paged latent cache for the given sequence lengths.
 
-    seqlens: list/1-D tensor of lengths (0 allowed).  Returns a PagedCache.
+    seqlens: list/1-D tensor of lengths (0 allowed).  s_q: query tokens per
+    sequence (q is [B, s_q, Hq, Dk]).  Returns a PagedCache.
     """
     gen = torch.Generator(device="cpu").manual_seed(int(seed))
     seqlens = torch.as_tensor(seqlens, dtype=torch.int32).reshape(-1)
@@ -149,7 +150,7 @@ def paged_decode_inputs(B, Hq, Dk, seqlens, page_size, seed, max_pages_per_seq=N
     n_used = sum(pages_per_seq)
     max_pp = max(pages_per_seq + [1]) if max_pages_per_seq is None else int(max_pages_per_seq)
     poison = n_used                      # index of the poison page
-    q = _randn_bf16(gen, (B, 1, Hq, Dk))
+    q = _randn_bf16(gen, (B, s_q, Hq, Dk))
     pool = _randn_bf16(gen, (n_used + 1, page_size, 1, Dk))
     sign = torch.randint(0, 2, (n_used + 1, page_size, 1, Dk), generator=gen) * 2 - 1
     sentinel = (sign.to(torch.float32) * SENTINEL).to(torch.bfloat16)

@@ -46,7 +46,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention", "decode_paged", "decode_paged_gqa", "gather_pages"]
+__all__ = ["attention", "decode_paged", "decode_paged_mtp", "decode_paged_gqa", "gather_pages"]
 
 
 def _rows_softmax_weighted(S: np.ndarray, V: np.ndarray):
@@ -190,4 +190,34 @@ def decode_paged_gqa(q, k_pages, v_pages, block_table, cache_seqlens, scale: flo
             o, lse = _rows_softmax_weighted(S, Vmat)
             O[i, heads] = o
             LSE[i, heads] = lse
+    return O, LSE
+
+
+def decode_paged_mtp(q, kv_pages, block_table, cache_seqlens, scale: float, dv: int, page_size: int = 64,
+                     seqs=None):
+    """MLA absorbed decode with s_q new query tokens per sequence.
+
+    q: [B, s_q, Hq, Dk].  The s_q query tokens are the last s_q cached tokens
+    of their sequence, so query token i of sequence b sees cached positions
+    0 .. L_b - s_q + i: the causal mask aligned to the bottom-right corner of
+    the dense formula (key j visible to query i iff j <= i + Nk - Nq, with
+    Nq = s_q, Nk = L_b).  K = the gathered latent rows, V = their first dv
+    entries, every head shares them (MQA-absorb form).  Returns O
+    [len(seqs), s_q, Hq, dv] and LSE [len(seqs), s_q, Hq] in fp64; a query
+    token with no visible position gets O = 0 and LSE = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kv_pages = np.asarray(kv_pages, dtype=np.float64)
+    B, sq, Hq, Dk = q.shape
+    bs = np.arange(B) if seqs is None else np.asarray(seqs, dtype=np.int64)
+    O = np.zeros((len(bs), sq, Hq, dv), dtype=np.float64)
+    LSE = np.full((len(bs), sq, Hq), -np.inf, dtype=np.float64)
+    for i, b in enumerate(bs):
+        L = int(cache_seqlens[b])
+        if L == 0:
+            continue
+        Kmat = gather_pages(kv_pages, block_table[b], L, page_size)
+        o, lse = attention(q[b][None], Kmat[None, :, None, :], Kmat[None, :, None, :dv], True, scale)
+        O[i] = o[0]
+        LSE[i] = lse[0].T
     return O, LSE
