@@ -19,8 +19,9 @@ import re
 
 import torch
 
-__all__ = ["fwd", "decode_paged", "decode_paged_noalloc", "decode_workspace_size", "decode_paged_gqa",
-           "decode_gqa_workspace_size", "read_device_status", "library", "AttnError", "exported_symbols", "STATUS"]
+__all__ = ["fwd", "decode_paged", "decode_paged_mtp", "decode_paged_noalloc", "decode_workspace_size",
+           "decode_mtp_workspace_size", "decode_paged_gqa", "decode_gqa_workspace_size", "read_device_status",
+           "library", "AttnError", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libattn_b200.so")
@@ -54,6 +55,8 @@ _SIGNATURES = {
     "attn_decode_paged_noalloc_max_bytes": (_sz, []),
     "attn_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "attn_decode_paged_gqa_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_decode_paged_mtp_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_decode_paged_mtp": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
 }
 
@@ -178,6 +181,50 @@ def decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Ten
                                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                          _stream_handle(q.device))
     _check(rc, "attn_decode_paged")
+    return out, lse
+
+
+def decode_mtp_workspace_size(B: int, s_q: int, Hq: int, Dv: int, device=None) -> int:
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(library().attn_decode_paged_mtp_workspace_size(B, s_q, Hq, Dv))
+
+
+def decode_paged_mtp(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
+                     scale: float, dv: int = 512, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None):
+    """Paged MLA decode with s_q query tokens per sequence (the last s_q cached
+    tokens; token i sees positions 0 .. L - s_q + i).
+
+    q [B,s_q,Hq,Dk] bf16; kv_pages [num_pages,page_size,1,Dk] bf16;
+    block_table [B,max_pages] int32; cache_seqlens [B] int32.
+    Returns (o [B,s_q,Hq,dv] bf16, lse [B,s_q,Hq] fp32).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kv_pages, "kv_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    B, sq, Hq, Dk = q.shape
+    num_pages, page_size, hkv, Dk2 = kv_pages.shape
+    if hkv != 1 or Dk2 != Dk or block_table.shape[0] != B or cache_seqlens.shape[0] != B:
+        raise ValueError("decode_paged_mtp shape mismatch")
+    if out is None:
+        out = torch.empty((B, sq, Hq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, sq, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    with torch.cuda.device(q.device):
+        need = int(library().attn_decode_paged_mtp_workspace_size(B, sq, Hq, dv))
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
+            raise ValueError("workspace too small")
+        rc = library().attn_decode_paged_mtp(q.data_ptr(), kv_pages.data_ptr(), block_table.data_ptr(),
+                                             cache_seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, sq, Hq, Dk,
+                                             dv, page_size, num_pages, block_table.shape[1], float(scale),
+                                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                             _stream_handle(q.device))
+    _check(rc, "attn_decode_paged_mtp")
     return out, lse
 
 

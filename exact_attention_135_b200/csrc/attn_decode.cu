@@ -82,18 +82,23 @@ constexpr int PREFETCH_PAGES = 2;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// The kernels work on query units: with s_q query tokens per sequence, unit
+// u = b * s_q + i is query token i of sequence b.  The s_q tokens are the last
+// s_q cached tokens, so unit u sees positions 0 .. L_b - s_q + i (the causal
+// mask aligned to the bottom-right corner) of block-table row b.
 struct Args {
-  const __nv_bfloat16* q;        // [B, Hq, DK]
+  const __nv_bfloat16* q;        // [B * s_q, Hq, DK]
   const uint8_t* kv;             // [num_pages, PAGE, DK] (only for L2 prefetches)
   const int32_t* block_table;    // [B, max_pages]
   const int32_t* seqlens;        // [B]
-  __nv_bfloat16* o;              // [B, Hq, DV]
-  float* lse;                    // [B, Hq]
-  int32_t* ws_pref;              // [B + 1]
+  __nv_bfloat16* o;              // [B * s_q, Hq, DV]
+  float* lse;                    // [B * s_q, Hq]
+  int32_t* ws_pref;              // [units + 1]
   float* ws_lse;                 // [2 * pairs, Hq]
   float* ws_o;                   // [2 * pairs, Hq, DV]
   int* status;
-  int B, max_pages, num_pages, pairs;
+  int B;                         // query units (sequences x s_q)
+  int s_q, max_pages, num_pages, pairs;
   float scale_log2;
 };
 
@@ -108,6 +113,13 @@ __device__ __forceinline__ int seq_len_eff(int L, int max_pages) {
   if (L <= 0) return 0;
   const int cap = max_pages * PAGE;
   return L < cap ? L : cap;
+}
+
+// Positions unit u attends to: its sequence's length clamped to the block
+// table, minus the query tokens after it.
+__device__ __forceinline__ int unit_len(const Args& a, int u) {
+  const int L = seq_len_eff(a.seqlens[u / a.s_q], a.max_pages) - (a.s_q - 1 - u % a.s_q);
+  return L > 0 ? L : 0;
 }
 
 // First page of pair p's range: floor(p * T / pairs).
@@ -194,8 +206,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int b = b0 + lane;
       int n = 0;
       if (b < a.B) {
-        const int L = a.seqlens[b];
-        n = seq_pages(L, a.max_pages);
+        const int L = a.seqlens[b / a.s_q];
+        n = seq_pages(unit_len(a, b), a.max_pages);
         bad |= (L < 0) || ((long long)L > (long long)a.max_pages * PAGE);
       }
       int x = n;   // inclusive warp scan
@@ -245,7 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (p_more) p_gp = p_g0;
       auto prefetch_next = [&]() {
         if (!p_more) return;
-        const int page = a.block_table[(size_t)p_b * a.max_pages + (p_gp - pref[p_b])];
+        const int page = a.block_table[(size_t)(p_b / a.s_q) * a.max_pages + (p_gp - pref[p_b])];
         if (page >= 0 && page < a.num_pages) l2_prefetch(a.kv + (size_t)page * STAGE_BYTES, STAGE_BYTES);
         if (++p_gp == p_g1) {
           p_more = wp.next(p_b, p_g0, p_g1);
@@ -259,7 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int ch = 0; ch < Q_SMEM_CHUNKS; ++ch)
           tma_load_2d(base + OFF_Q + ch * Q_CHUNK_BYTES, &tm_q, bar(B_QF), ch * 64, sb * HQ);
         q_last = seg;
-        const int32_t* row = a.block_table + (size_t)sb * a.max_pages;
+        const int32_t* row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages;
         for (int gp = g0; gp < g1; ++gp, ++g) {
           int page = row[gp - pref[sb]];
           if (page < 0 || page >= a.num_pages) {
@@ -393,7 +405,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_QT));
       }
-      const int L = seq_len_eff(a.seqlens[sb], a.max_pages);
+      const int L = unit_len(a, sb);
       const int first_page = pref[sb];
       float m_run = -INFINITY, l_run = 0.f;
       for (int gp = g0; gp < g1; ++gp, ++g) {
@@ -589,34 +601,40 @@ inline int pairs_for_device() {
 }  // namespace dec
 }  // namespace ea
 
-extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv) {
+extern "C" size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv) {
   using namespace ea::dec;
-  if (B < 1 || B > B_MAX || Hq != HQ || Dv != DV) return 0;
+  if (B < 1 || s_q < 1 || (long long)B * s_q > B_MAX || Hq != HQ || Dv != DV) return 0;
   const int pairs = pairs_for_device();
   if (pairs == 0) return 0;
-  return ws_layout(B, pairs).total;
+  return ws_layout(B * s_q, pairs).total;
 }
 
-extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_table,
-                                 const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk, int Dv,
-                                 int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv) {
+  return attn_decode_paged_mtp_workspace_size(B, 1, Hq, Dv);
+}
+
+extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const int32_t* block_table,
+                                     const int32_t* cache_seqlens, void* o, float* lse, int B, int s_q, int Hq, int Dk,
+                                     int Dv, int page_size, int num_pages, int max_pages_per_seq, float scale,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
   using namespace ea;
   using namespace ea::dec;
   if (!q || !kv_pages || !block_table || !cache_seqlens || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(kv_pages, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(block_table, 4) || !aligned(cache_seqlens, 4))
     return ATTN_ERR_INVALID_ARG;
-  if (B < 1 || num_pages < 1 || max_pages_per_seq < 1 || page_size < 1 || Hq < 1 || Dk < 1 || Dv < 1)
+  if (B < 1 || s_q < 1 || num_pages < 1 || max_pages_per_seq < 1 || page_size < 1 || Hq < 1 || Dk < 1 || Dv < 1)
     return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (Hq != HQ || Dk != DK || Dv != DV || page_size != PAGE || B > B_MAX) return ATTN_ERR_UNSUPPORTED;
+  if (Hq != HQ || Dk != DK || Dv != DV || page_size != PAGE || (long long)B * s_q > B_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  const int units = B * s_q;
   if ((long long)num_pages * PAGE >= (1ll << 31) || (long long)B * max_pages_per_seq >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
   const int pairs = pairs_for_device();
   if (pairs == 0) return ATTN_ERR_CUDA;
   if (pairs > MAX_PARTS) return ATTN_ERR_UNSUPPORTED;
-  const WsLayout wl = ws_layout(B, pairs);
+  const WsLayout wl = ws_layout(units, pairs);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
 
   static int attr_done = 0;
@@ -627,7 +645,7 @@ extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int3
 
   CUtensorMap tq, tkv;
   {
-    const uint64_t dims[2] = {(uint64_t)DK, (uint64_t)B * HQ};
+    const uint64_t dims[2] = {(uint64_t)DK, (uint64_t)units * HQ};
     const uint64_t strides[1] = {(uint64_t)DK * 2};
     const uint32_t box[2] = {64, (uint32_t)HQ};
     if (!encode_bf16_2d(&tq, q, dims, strides, box)) return ATTN_ERR_CUDA;
@@ -650,7 +668,8 @@ extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int3
   a.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
   a.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
   a.status = status;
-  a.B = B;
+  a.B = units;
+  a.s_q = s_q;
   a.max_pages = max_pages_per_seq;
   a.num_pages = num_pages;
   a.pairs = pairs;
@@ -658,8 +677,16 @@ extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int3
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   decode_split_kernel<<<2 * pairs, THREADS, SMEM_BYTES, s>>>(tq, tkv, a);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  decode_combine_kernel<<<dim3(B, HQ / COMBINE_HEADS), COMBINE_THREADS, 0, s>>>(a);
+  decode_combine_kernel<<<dim3(units, HQ / COMBINE_HEADS), COMBINE_THREADS, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_table,
+                                 const int32_t* cache_seqlens, void* o, float* lse, int B, int Hq, int Dk, int Dv,
+                                 int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return attn_decode_paged_mtp(q, kv_pages, block_table, cache_seqlens, o, lse, B, 1, Hq, Dk, Dv, page_size,
+                               num_pages, max_pages_per_seq, scale, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -124,6 +124,35 @@ int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_
                       size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_paged_mtp_workspace_size: workspace bytes of attn_decode_paged_mtp
+ * for B sequences with s_q query tokens each (0 for an unsupported shape).
+ */
+size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv);
+
+/*
+ * attn_decode_paged_mtp: attn_decode_paged with s_q >= 1 new query tokens per
+ * sequence (multi-token prediction / speculative decoding; "GQLA ..." page,
+ * MTP with the MQA-absorb path).  The s_q query tokens are the last s_q cached
+ * tokens of their sequence (their latent rows are already in the cache), so
+ * query token i sees cached positions 0 .. L_b - s_q + i: the causal mask of
+ * attn_fwd, aligned to the bottom-right corner.  A token with no visible
+ * position gets O = 0 and LSE = -inf.
+ *
+ *   q    [B, s_q, Hq, Dk] bf16      o   [B, s_q, Hq, Dv] bf16 (written)
+ *   lse  [B, s_q, Hq] fp32 (written)
+ *
+ * Every other argument, layout and error is that of attn_decode_paged, whose
+ * call equals this one with s_q = 1.  Supported: B * s_q <= 2048.  Each query
+ * token is scheduled as its own unit over the sequence's block-table row (the
+ * fp32 accumulator of 128 heads x 512 already fills an SM's tensor memory, so
+ * query tokens are not stacked into one MMA tile).
+ */
+int attn_decode_paged_mtp(const void* q, const void* kv_pages, const int32_t* block_table,
+                          const int32_t* cache_seqlens, void* o, float* lse, int B, int s_q, int Hq, int Dk, int Dv,
+                          int page_size, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_paged_noalloc: attn_decode_paged without a caller workspace.
  * The source pages describe no counterpart of this entry point; it exists for
  * callers that cannot allocate device memory at decode time (a serving engine

@@ -98,3 +98,14 @@ def test_gqa_decode_unsupported_shapes(lib):
     assert _gqa(lib, Hq=32, Hkv=2) == 2      # group of 16
     assert _gqa(lib, page=16) == 2
     assert _gqa(lib, B=5000) == 2
+
+
+def test_mtp_decode_argument_checks(lib):
+    def call(B=2, s_q=2, Hq=128, Dk=576, Dv=512, page=64, q=A, scale=0.07):
+        return lib.attn_decode_paged_mtp(q, A, A, A, A, A, B, s_q, Hq, Dk, Dv, page, 8, 4, scale, A, 1 << 20, None)
+    assert call(q=None) == 1
+    assert call(s_q=0) == 1
+    assert call(scale=-1.0) == 1
+    assert call(Hq=64) == 2
+    assert call(B=1024, s_q=4) == 2          # more than 2048 query units
+    assert lib.attn_decode_paged_mtp_workspace_size(1024, 4, 128, 512) == 0
