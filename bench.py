@@ -205,6 +205,39 @@ def decode_part(ea, dev):
     return p
 
 
+MTP_SQ = 2   # query tokens per sequence of the multi-token decode part
+
+
+def mtp_part(ea, dev):
+    cfg = inputs.DECODE_CONFIG
+    gen = torch.Generator(device="cpu").manual_seed(int(cfg.seed))
+    lens = torch.randint(cfg.min_len, cfg.max_len + 1, (cfg.B,), generator=gen, dtype=torch.int32)
+    c = inputs.paged_decode_inputs(cfg.B, cfg.Hq, cfg.Dk, lens, cfg.page_size, cfg.seed + 200000, s_q=MTP_SQ)
+    host = {"q": c.q.pin_memory(), "kv": c.kv_pages.pin_memory(), "bt": c.block_table.pin_memory(),
+            "sl": c.cache_seqlens.pin_memory()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    d["o"] = torch.empty((cfg.B, MTP_SQ, cfg.Hq, cfg.Dv), dtype=torch.bfloat16, device=dev)
+    d["lse"] = torch.empty((cfg.B, MTP_SQ, cfg.Hq), dtype=torch.float32, device=dev)
+    d["ws"] = torch.empty(ea.decode_mtp_workspace_size(cfg.B, MTP_SQ, cfg.Hq, cfg.Dv, dev), dtype=torch.uint8,
+                          device=dev)
+    host["o"] = torch.empty(d["o"].shape, dtype=torch.bfloat16).pin_memory()
+    host["lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
+
+    def run():
+        ea.decode_paged_mtp(d["q"], d["kv"], d["bt"], d["sl"], cfg.scale, dv=cfg.Dv, out=d["o"], lse=d["lse"],
+                            workspace=d["ws"])
+
+    p = Part("mtp", run, [(d[n], host[n]) for n in ("q", "kv", "bt", "sl")],
+             [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=2)
+    p.cfg = cfg
+    p.kv_bytes = c.kv_valid_bytes(cfg.Dk)
+    p.tokens = int(c.cache_seqlens.to(torch.int64).sum())
+    # query token i of a sequence of length L attends to L - s_q + 1 + i positions
+    p.pairs = MTP_SQ * p.tokens - cfg.B * MTP_SQ * (MTP_SQ - 1) // 2
+    p.flops = 2.0 * cfg.Hq * (cfg.Dk + cfg.Dv) * p.pairs
+    return p
+
+
 def gqa_part(ea, dev):
     cfg = inputs.GQA_DECODE_CONFIG
     c = inputs.gqa_decode_config_inputs(cfg)
@@ -290,6 +323,8 @@ def run_gpu(args):
         parts.append(decode_part(ea, dev))
     if args.part in ("all", "gqa"):
         parts.append(gqa_part(ea, dev))
+    if args.part in ("all", "mtp"):
+        parts.append(mtp_part(ea, dev))
 
     for _ in range(args.warmup):
         for p in parts:
@@ -368,6 +403,25 @@ def run_gpu(args):
                     "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
             "workspace_bytes": p.ws_bytes,
         }
+    mtp_obj = None
+    if "mtp" in by:
+        p = by["mtp"]
+        sec = launch_ms["mtp"] * 1e-3
+        mtp_obj = {
+            "metric": f"KV-cache GB/s (paged MLA decode, {MTP_SQ} query tokens per sequence)",
+            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["mtp"]) / 1e9, 1), "unit": "GB/s",
+            "ms_per_launch": round(launch_ms["mtp"], 4),
+            "query_tokens_per_s": round(world * p.cfg.B * MTP_SQ / sec, 1),
+            "config": {"workload": p.cfg.name + f", s_q={MTP_SQ}", "s_q": MTP_SQ, "kv_bytes": p.kv_bytes,
+                       "attended_positions": p.pairs},
+            "roofline": {"bound": "hbm", "achieved": round(p.kv_bytes / sec / 1e9, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(p.kv_bytes / sec / 1e9 / peaks["hbm_gbs"], 4),
+                         "peak_kind": f"{peaks_kind} HBM copy", "traffic": None,
+                         "kernel": "decode_split_kernel + decode_combine_kernel (query units)",
+                         "tflops": round(p.flops / sec / 1e12, 1)},
+            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["mtp"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+        }
     if "prefill" in by:
         p = by["prefill"]
         achieved = p.work / (launch_ms["prefill"] * 1e-3) / 1e12
@@ -395,8 +449,10 @@ def run_gpu(args):
             line["decode"] = decode_obj
         if gqa_obj:
             line["gqa_decode"] = gqa_obj
+        if mtp_obj:
+            line["decode_mtp"] = mtp_obj
     else:
-        head = decode_obj if decode_obj else gqa_obj
+        head = decode_obj or gqa_obj or mtp_obj
         line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
         line["config"]["step"] = step_parts
         if decode_obj and gqa_obj:
@@ -499,7 +555,7 @@ def main():
     ap.add_argument("--baseline-rows", type=int, default=768,
                     help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa"], default="all",
+    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp"], default="all",
                     help="time only one piece of the step (for profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()
