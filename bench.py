@@ -51,7 +51,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
     "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
-    "decode": 349399808 + 16235008,     # decode_split_kernel, MLA decode workload
+    "decode": 349649664 + 16860928,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
 }
 # Timed regions longer than this run under the power cap: compare with the
