@@ -39,7 +39,9 @@ chunk holds complete rows of S, so no online rescaling takes place.
 
 Parity pins: tests/test_oracle.py checks this module against hand-derived
 values (tests/golden/), closed forms, invariants, a pure-Python brute force
-and torch's fp64 scaled_dot_product_attention.
+and torch's fp64 scaled_dot_product_attention; tests/test_oracle_gqa.py and
+tests/test_oracle_mtp.py pin the GQA-path and multi-token decode functions
+with brute forces, closed forms, invariances and planted mistakes.
 """
 
 from __future__ import annotations
