@@ -155,3 +155,27 @@ def test_workspace_checks():
                                lse.data_ptr(), 2, HQ, DK, DV, PAGE, kv.shape[0], bt.shape[1], SCALE,
                                small.data_ptr(), need - 256, None)
     assert rc == 5   # ATTN_ERR_WORKSPACE
+
+
+def test_maximum_batch_of_sequences():
+    """B = 2048, the largest batch the split plan holds in shared memory:
+    2048 short sequences (0..40 tokens, so most pages are cut), checked on a
+    sample of sequences against the oracle; the rest must be finite."""
+    rng = np.random.default_rng(31)
+    lens = rng.integers(0, 41, size=2048).tolist()
+    c = inputs.paged_decode_inputs(len(lens), HQ, DK, lens, PAGE, seed=31)
+    o, lse = _run(c)
+    assert ea.read_device_status(0) == 0
+    seqs = [0, 1, 511, 1024, 1500, 2047] + [int(np.argmax(lens))]
+    o_ref, lse_ref = _oracle(c, seqs)
+    compare(o[seqs, 0], lse[seqs], o_ref, lse_ref, "MLA decode B=2048", o_max_abs=bf16_arith_bound(_valid_vmax(c)))
+    assert torch.isfinite(o).all()
+    empty = torch.tensor(lens) == 0
+    assert torch.isneginf(lse.cpu()[empty]).all() and torch.isfinite(lse.cpu()[~empty]).all()
+
+
+def test_batch_above_maximum_is_rejected():
+    c = inputs.paged_decode_inputs(2049, HQ, DK, [1] * 2049, PAGE, seed=2)
+    with pytest.raises(ea.AttnError) as e:
+        _run(c)
+    assert e.value.code == 2

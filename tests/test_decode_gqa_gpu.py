@@ -140,3 +140,19 @@ def test_workspace_too_small_is_rejected():
     assert lib.attn_decode_paged_gqa(*args, need, stream) == 0
     torch.cuda.synchronize()
     assert ea.read_device_status(0) == 0
+
+
+def test_maximum_batch_of_sequences():
+    """B = 2048 short sequences (0..70 tokens), groups of 8: the largest batch."""
+    rng = np.random.default_rng(41)
+    lens = rng.integers(0, 71, size=2048).tolist()
+    c = inputs.paged_gqa_decode_inputs(len(lens), 8, 1, 128, lens, PAGE, 41)
+    o, lse = _run(c, 0.0883883)
+    assert ea.read_device_status(0) == 0
+    seqs = [0, 3, 777, 1024, 2047, int(np.argmax(lens))]
+    o_ref, lse_ref = oracle.decode_paged_gqa(to_np64(c.q)[:, 0], to_np64(c.k_pages), to_np64(c.v_pages),
+                                             c.block_table.numpy(), c.cache_seqlens.numpy(), 0.0883883,
+                                             page_size=PAGE, seqs=seqs)
+    compare(o[seqs, 0], lse[seqs], o_ref, lse_ref, "gqa decode B=2048", o_max_abs=bf16_arith_bound(_vmax(c)))
+    empty = torch.tensor(lens) == 0
+    assert torch.isneginf(lse.cpu()[empty]).all() and torch.isfinite(lse.cpu()[~empty]).all()

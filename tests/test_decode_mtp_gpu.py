@@ -77,3 +77,15 @@ def test_two_tokens_on_the_decode_workload_sampled():
     seqs = [0, 9, 21, 40, 55, 63]
     o_ref, lse_ref = _oracle(c, seqs=seqs)
     compare(o[seqs], lse[seqs], o_ref, lse_ref, "mtp decode workload 5, s_q=2 (sampled sequences)")
+
+
+def test_maximum_query_units():
+    """B * s_q = 2048 query units (512 sequences x 4 tokens), short sequences."""
+    rng = np.random.default_rng(51)
+    lens = rng.integers(0, 90, size=512).tolist()
+    c = inputs.paged_decode_inputs(len(lens), HQ, DK, lens, PAGE, seed=51, s_q=4)
+    o, lse = _run(c)
+    assert ea.read_device_status(0) == 0
+    seqs = [0, 100, 255, 511, int(np.argmax(lens))]
+    o_ref, lse_ref = _oracle(c, seqs=seqs)
+    compare(o[seqs], lse[seqs], o_ref, lse_ref, "mtp decode 2048 query units", o_max_abs=bf16_arith_bound(_vmax(c)))
