@@ -29,6 +29,10 @@ What it computes is the plain definition the fused kernels must reach exactly
   of query heads reads its own group-expanded cache.  Here that is a paged
   cache of separate K and V rows per (token, KV head); query head h reads KV
   head h // (Hq / Hkv), as in the dense oracle.
+* "Flash Attention" wiki page, section "구조화된 지식 (Synthesized Content)",
+  item "Recomputation (재계산)": the backward pass recomputes the intermediate
+  matrices instead of storing them.  ``attention_bwd`` writes out the plain
+  derivative of the forward definition (dQ, dK, dV for an upstream dO).
 
 Outputs: O (fp64) and LSE = ln sum_j exp(S_ij) (fp64, natural log of the sum
 over the *scaled* scores).  A row with no visible key has O = 0, LSE = -inf.
@@ -41,14 +45,17 @@ Parity pins: tests/test_oracle.py checks this module against hand-derived
 values (tests/golden/), closed forms, invariants, a pure-Python brute force
 and torch's fp64 scaled_dot_product_attention; tests/test_oracle_gqa.py and
 tests/test_oracle_mtp.py pin the GQA-path and multi-token decode functions
-with brute forces, closed forms, invariances and planted mistakes.
+with brute forces, closed forms, invariances and planted mistakes;
+tests/test_oracle_bwd.py pins the gradients with central finite differences
+of the forward function, torch fp64 autograd, closed forms, the zero sum of
+the dK rows and planted mistakes.
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention", "decode_paged", "decode_paged_mtp", "decode_paged_gqa", "gather_pages"]
+__all__ = ["attention", "attention_bwd", "decode_paged", "decode_paged_mtp", "decode_paged_gqa", "gather_pages"]
 
 
 def _rows_softmax_weighted(S: np.ndarray, V: np.ndarray):
@@ -223,3 +230,79 @@ def decode_paged_mtp(q, kv_pages, block_table, cache_seqlens, scale: float, dv: 
         O[i] = o[0]
         LSE[i] = lse[0].T
     return O, LSE
+
+
+def attention_bwd(q, k, v, do, causal: bool, scale: float, q_rows=None, k_rows=None, kv_heads=None,
+                  row_chunk: int = 1024):
+    """Gradients of exact attention with respect to Q, K and V.
+
+    "Flash Attention" wiki page, section "구조화된 지식 (Synthesized Content)",
+    item "Recomputation (재계산)": the backward pass does not keep the N x N
+    intermediate matrices; it recomputes what it needs from the inputs.  The
+    page gives no formulas.  What the backward must reach is the plain
+    derivative of the forward definition (the one in ``attention``), which is
+    what this function writes out, S and P materialised one block of complete
+    rows at a time.  For one (batch, query head) with KV head kv and upstream
+    gradient dO = dL/dO:
+
+        S = scale * Q K^T (causal: -inf where key j > i + Nk - Nq)
+        P = softmax of each row of S          (a row with no visible key: 0)
+        dV_kv += P^T dO
+        dP = dO V^T
+        dS = P * (dP - rowsum(P * dP))          (softmax Jacobian, row by row)
+        dQ = scale * dS K
+        dK_kv += scale * dS^T Q
+
+    dK and dV of a KV head sum over every query head of its group.
+
+    q: [B, Nq, Hq, D]; k: [B, Nk, Hkv, D]; v: [B, Nk, Hkv, Dv]; do: [B, Nq, Hq, Dv].
+    q_rows / k_rows: optional index arrays; dQ is returned for those query rows
+    and dK, dV for those key rows only (every query row still enters dK and
+    dV, so the cost stays that of the full problem).  kv_heads: optional
+    subset of KV heads; only their query heads are computed, the other heads'
+    entries stay 0.  Returns dQ [B, len(q_rows), Hq, D], dK [B, len(k_rows),
+    Hkv, D], dV [B, len(k_rows), Hkv, Dv] in fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, _ = k.shape
+    Dv = v.shape[3]
+    assert do.shape == (B, Nq, Hq, Dv) and Hq % Hkv == 0
+    group = Hq // Hkv
+    qr = np.arange(Nq) if q_rows is None else np.asarray(q_rows, dtype=np.int64)
+    kr = np.arange(Nk) if k_rows is None else np.asarray(k_rows, dtype=np.int64)
+    heads_kv = range(Hkv) if kv_heads is None else [int(h) for h in kv_heads]
+    dQ = np.zeros((B, len(qr), Hq, D))
+    dK = np.zeros((B, len(kr), Hkv, D))
+    dV = np.zeros((B, len(kr), Hkv, Dv))
+    if Nk == 0 or Nq == 0:
+        return dQ, dK, dV
+    q_pos = {int(r): i for i, r in enumerate(qr)}
+    key_idx = np.arange(Nk)
+    for b in range(B):
+        for kv in heads_kv:
+            Kmat = k[b, :, kv, :]
+            Vmat = v[b, :, kv, :]
+            for hq in range(kv * group, (kv + 1) * group):
+                for r0 in range(0, Nq, row_chunk):
+                    rows = np.arange(r0, min(Nq, r0 + row_chunk))
+                    S = scale * (q[b, rows, hq, :] @ Kmat.T)
+                    if causal:
+                        S = np.where(key_idx[None, :] <= rows[:, None] + (Nk - Nq), S, -np.inf)
+                    m = np.max(S, axis=1, keepdims=True)
+                    m = np.where(np.isfinite(m), m, 0.0)
+                    E = np.exp(S - m)
+                    l = np.sum(E, axis=1, keepdims=True)
+                    P = np.divide(E, l, out=np.zeros_like(E), where=l > 0)
+                    dOr = do[b, rows, hq, :]
+                    dP = dOr @ Vmat.T
+                    dS = P * (dP - np.sum(P * dP, axis=1, keepdims=True))
+                    dV[b, :, kv, :] += P[:, kr].T @ dOr
+                    dK[b, :, kv, :] += scale * (dS[:, kr].T @ q[b, rows, hq, :])
+                    sel = [i for i, r in enumerate(rows) if int(r) in q_pos]
+                    if sel:
+                        dQ[b, [q_pos[int(rows[i])] for i in sel], hq, :] = scale * (dS[sel] @ Kmat)
+    return dQ, dK, dV
