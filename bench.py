@@ -11,7 +11,10 @@ already resident in device memory:
     uniform on [1024, 8192]);
   * gqa:     attn_decode_paged_gqa on the GQA-path paged-decode workload
     (64 sequences x 32 query heads in 8 groups, D=128, separate K/V pages,
-    the same length mix).
+    the same length mix);
+  * mtp:     attn_decode_paged_mtp, the MLA decode with two query tokens per
+    sequence;
+  * bwd:     attn_bwd (gradients of the prefill) on the long-context workload.
 The headline metric is prefill TFLOP/s (4*Nq*Nk*D per head, halved for
 causal); the decode KV-cache GB/s (bytes of the K/V rows of valid tokens
 over the time of the decode + combine kernels) is reported in the "decode"
@@ -53,6 +56,7 @@ NCU_TRAFFIC_BYTES = {
     "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
     "decode": 349649664 + 16860928,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
+    "bwd": None,                        # attn_bwd_kernel<D=128, causal>: not captured yet
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.
@@ -265,6 +269,34 @@ def gqa_part(ea, dev):
     return p
 
 
+def bwd_part(ea, dev):
+    """attn_bwd on the long-context GQA causal workload: O and LSE come from
+    one forward pass at setup; dO ~ N(0,1) bf16 from its own seeded stream."""
+    cfg = inputs.PREFILL_CONFIGS[PREFILL_ID]
+    q, k, v, do = inputs.bwd_config_inputs(cfg)
+    host = {"q": q.pin_memory(), "k": k.pin_memory(), "v": v.pin_memory(), "do": do.pin_memory()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    d["o"], d["lse"] = ea.fwd(d["q"], d["k"], d["v"], causal=cfg.causal, scale=cfg.scale)
+    host["o"] = d["o"].cpu().pin_memory()
+    host["lse"] = d["lse"].cpu().pin_memory()
+    for n, ref in (("dq", "q"), ("dk", "k"), ("dv", "v")):
+        d[n] = torch.empty_like(d[ref])
+        host[n] = torch.empty(d[n].shape, dtype=torch.bfloat16).pin_memory()
+    d["ws"] = torch.empty(ea.bwd_workspace_size(cfg.B, cfg.Hq, cfg.Nq, cfg.D), dtype=torch.uint8, device=dev)
+
+    def run():
+        ea.bwd(d["q"], d["k"], d["v"], d["o"], d["lse"], d["do"], causal=cfg.causal, scale=cfg.scale,
+               dq=d["dq"], dk=d["dk"], dv=d["dv"], workspace=d["ws"])
+
+    p = Part("bwd", run, [(d[n], host[n]) for n in ("q", "k", "v", "o", "lse", "do")],
+             [(host[n], d[n]) for n in ("dq", "dk", "dv")], launches=3)
+    p.cfg = cfg
+    # five products of the size of one forward product pair: 2.5 x the forward count
+    p.work = 2.5 * cfg.flops()
+    p.ws_bytes = d["ws"].numel()
+    return p
+
+
 def time_parts(parts, steps, stream):
     """Times `steps` steps; each step runs every part once.  Returns total ms
     and per-part lists of per-launch ms (CUDA events on the launching stream)."""
@@ -325,6 +357,8 @@ def run_gpu(args):
         parts.append(gqa_part(ea, dev))
     if args.part in ("all", "mtp"):
         parts.append(mtp_part(ea, dev))
+    if args.part in ("all", "bwd"):
+        parts.append(bwd_part(ea, dev))
 
     for _ in range(args.warmup):
         for p in parts:
@@ -422,6 +456,26 @@ def run_gpu(args):
             "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["mtp"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
         }
+    sustained = step_ms * args.steps * 1e-3 > SUSTAINED_AFTER_S
+    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    bf16_kind = f"{peaks_kind} bf16 {'sustained' if sustained else 'burst'}"
+    bwd_obj = None
+    if "bwd" in by:
+        p = by["bwd"]
+        tf = p.work / (launch_ms["bwd"] * 1e-3) / 1e12
+        bwd_obj = {
+            "metric": "attention backward TFLOP/s",
+            "value": round(whole_job_rate(world, p.work, launch_ms["bwd"]) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_launch": round(launch_ms["bwd"], 4),
+            "config": {"workload": "backward of " + p.cfg.name, "flops": "2.5 x forward (five products)",
+                       "workspace_bytes": p.ws_bytes},
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": round(tf / bf16_peak, 4), "peak_kind": bf16_kind, "traffic": NCU_TRAFFIC_BYTES["bwd"],
+                         "kernel": "bwd_prep_kernel + attn_bwd_kernel<D=128,causal> + bwd_dq_kernel (timed together)",
+                         "frac_of_burst": round(tf / peaks["bf16_tflops"], 4)},
+            "e2e": {"value": round(world * p.work / (e2e_ms["bwd"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+        }
     if "prefill" in by:
         p = by["prefill"]
         achieved = p.work / (launch_ms["prefill"] * 1e-3) / 1e12
@@ -451,8 +505,10 @@ def run_gpu(args):
             line["gqa_decode"] = gqa_obj
         if mtp_obj:
             line["decode_mtp"] = mtp_obj
+        if bwd_obj:
+            line["bwd"] = bwd_obj
     else:
-        head = decode_obj or gqa_obj or mtp_obj
+        head = decode_obj or gqa_obj or mtp_obj or bwd_obj
         line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
         line["config"]["step"] = step_parts
         if decode_obj and gqa_obj:
@@ -555,7 +611,7 @@ def main():
     ap.add_argument("--baseline-rows", type=int, default=768,
                     help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp"], default="all",
+    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp", "bwd"], default="all",
                     help="time only one piece of the step (for profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()

@@ -58,6 +58,8 @@ _SIGNATURES = {
     "attn_decode_paged_mtp_workspace_size": (_sz, [_i, _i, _i, _i]),
     "attn_decode_paged_mtp": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_bwd": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _sz, _vp]),
 }
 
 
@@ -139,6 +141,49 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                                 _stream_handle(q.device))
     _check(rc, "attn_fwd")
     return out, lse
+
+
+def bwd_workspace_size(B: int, Hq: int, Nq: int, D: int) -> int:
+    return int(library().attn_bwd_workspace_size(B, Hq, Nq, D))
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+        causal: bool = False, scale: float | None = None, dq: torch.Tensor | None = None,
+        dk: torch.Tensor | None = None, dv: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Gradients of ``fwd`` with respect to q, k, v for the upstream gradient dout.
+
+    q, o, dout [B,Nq,Hq,D]; k, v [B,Nk,Hkv,D] bf16; lse [B,Hq,Nq] fp32 from
+    ``fwd`` on the same inputs.  Returns (dq, dk, dv) bf16 with the shapes of
+    q, k, v.  Runs on torch's current stream of q's device.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, Nq, Hq, D = q.shape
+    _, Nk, Hkv, _ = k.shape
+    Dv = v.shape[3]
+    if (tuple(k.shape) != (B, Nk, Hkv, D) or tuple(v.shape[:3]) != (B, Nk, Hkv) or o.shape != dout.shape
+            or tuple(o.shape) != (B, Nq, Hq, Dv) or tuple(lse.shape) != (B, Hq, Nq)):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _need(t, n, torch.bfloat16, 4)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape mismatch")
+    need = bwd_workspace_size(B, Hq, Nq, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        rc = library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk,
+                                D, Dv, int(bool(causal)), float(scale), workspace.data_ptr(), workspace.numel(),
+                                _stream_handle(q.device))
+    _check(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def decode_workspace_size(B: int, Hq: int, Dv: int, device=None) -> int:

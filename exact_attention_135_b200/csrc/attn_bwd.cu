@@ -1,0 +1,645 @@
+// Exact-attention backward pass for sm_100a (B200), with recomputation.
+//
+// What it computes ("Flash Attention" wiki page, section "구조화된 지식
+// (Synthesized Content)", item "Recomputation (재계산)": the backward pass
+// recomputes the intermediate matrices instead of reading stored N x N ones):
+// the gradients of O = softmax(scale * Q K^T + causal mask) V for an upstream
+// gradient dO, with S and P rebuilt block by block from Q, K and the forward's
+// LSE.  For one query head and its KV head:
+//
+//   P  = exp(scale * Q K^T - LSE)            (0 where masked)
+//   dV = P^T dO        dP = dO V^T           Drow = rowsum(dO * O)
+//   dS = P * (dP - Drow)
+//   dQ = scale * dS K  dK = scale * dS^T Q   (dK, dV summed over the group's heads)
+//
+// Drow equals rowsum(P * dP) because O = P V, which is what makes the softmax
+// Jacobian cheap.  Three launches:
+//
+//   bwd_prep_kernel   Drow (fp32) from O and dO, and a zeroed fp32 dQ accumulator
+//   attn_bwd_kernel   one CTA per (key block of 128, KV head, batch).  dK and dV
+//                     stay in TMEM while the CTA walks every query block of
+//                     every query head of the group that sees its keys; each
+//                     step's dQ contribution is added to the accumulator
+//   bwd_dq_kernel     dQ accumulator -> bf16
+//
+// Roles inside attn_bwd_kernel (320 threads, 200 registers each):
+//   warps 0-3  (WG0)  one key row per thread: S^T, dP^T from TMEM, P and dS -> bf16
+//                     into TMEM (for dV, dK) and dS into shared memory (for dQ)
+//   warps 4-7  (WG1)  one query row per thread: dQ from TMEM -> fp32 atomics;
+//                     at the end dK, dV -> bf16 -> global
+//   warp 8            TMA: K, V once; a two-stage ring of (Q, dO) tiles plus the
+//                     step's LSE and Drow values
+//   warp 9            tcgen05.mma issue
+//
+// TMEM (128 lanes x 512 fp32 columns): dV [0, D), dK [D, 2D), region A
+// [2D, 2D+128) = S^T then P^T (bf16, first 64 columns), region B
+// [2D+128, 2D+256) = dP^T then dS^T (bf16, first 64 columns) then dQ.  Issue
+// order per step i (tcgen05.mma executes in issue order, so an MMA may
+// overwrite columns an earlier one reads):
+//   dV_i (reads P^T_i) -> S^T_{i+1} (A) -> dK_i (reads dS^T_i) -> dQ_i (B)
+//   -> [dQ_i drained by WG1] -> dP^T_{i+1} (B)
+// so the next step's S^T is computed while WG0 still forms dS_i, and dQ's
+// drain overlaps the next step's softmax work.
+#include <math.h>
+
+#include "host_common.h"
+#include "sm100.cuh"
+
+namespace ea {
+namespace bwd {
+
+template <int D_, bool CAUSAL_>
+struct Cfg {
+  static constexpr int D = D_;
+  static constexpr bool CAUSAL = CAUSAL_;
+  static constexpr int BM = 128;                   // query rows per step
+  static constexpr int BN = 128;                   // keys per CTA = TMEM lanes
+  static constexpr int DCH = D / 64;               // 128-byte column chunks of a tile
+  static constexpr int CH = 128 * 128;             // bytes of one chunk of a 128-row tile
+  static constexpr int TILE = 128 * D * 2;         // bytes of one 128-row bf16 tile
+  static constexpr int DS_BYTES = BM * BN * 2;     // dS tile, A operand of dQ (MN-major)
+  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_DS = OFF_V + TILE;
+  static constexpr int OFF_STAGE = OFF_DS + DS_BYTES;   // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
+  static constexpr int OFF_ROWS = OFF_STAGE + 4 * TILE;  // stage s: lse2[128], drow[128] at +s*1024
+  static constexpr int OFF_BAR = OFF_ROWS + 2 * 1024;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1;        // [2] stage full (TMA bytes + producer arrival)
+  static constexpr int B_QE = 3;        // [2] stage empty (MMA commit)
+  static constexpr int B_SF = 5;        // S^T in TMEM
+  static constexpr int B_DPF = 6;       // dP^T in TMEM
+  static constexpr int B_DQF = 7;       // dQ in TMEM
+  static constexpr int B_PR = 8;        // P^T stored (4 WG0 warps)
+  static constexpr int B_DSR = 9;       // dS stored in TMEM and shared memory (4 WG0 warps)
+  static constexpr int B_DQE = 10;      // dQ drained (4 WG1 warps)
+  static constexpr int B_DONE = 11;     // every MMA of the CTA complete
+  static constexpr int NBAR = 12;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int LAYOUT_BYTES = OFF_MISC + 16;
+  static constexpr int MAX_SMEM = 227 * 1024;
+  // Room for re-aligning the dynamic shared-memory base when it fits; the
+  // kernel checks the alignment it got against what it was given.
+  static constexpr int SMEM_BYTES = LAYOUT_BYTES + 1024 <= MAX_SMEM ? LAYOUT_BYTES + 1024 : MAX_SMEM;
+  static_assert(LAYOUT_BYTES <= MAX_SMEM, "shared memory budget");
+  // TMEM columns
+  static constexpr int DV_COL = 0;
+  static constexpr int DK_COL = D;
+  static constexpr int A_COL = 2 * D;
+  static constexpr int B_COL = 2 * D + 128;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(B_COL + 128 <= TMEM_COLS, "TMEM budget");
+  // Ten warps: the register file is split per SM sub-partition, so the
+  // sub-partitions holding three warps cap every thread at 168 registers.
+  static constexpr int THREADS = 320;
+  static constexpr int PRODUCER_WARP = 8;
+  static constexpr int MMA_WARP = 9;
+};
+
+struct Args {
+  const float* lse;      // [B, Hq, Nq] natural log
+  const float* drow;     // [B, Hq, Nq]
+  float* dq_acc;         // [B, Nq, Hq, D]
+  __nv_bfloat16* dk;     // [B, Nk, Hkv, D]
+  __nv_bfloat16* dv;     // [B, Nk, Hkv, D]
+  int* status;
+  int B, Hq, Hkv, Nq, Nk, group, n_qblk, n_kblk, causal_off;
+  float scale, scale_log2;
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const Args a) {
+  constexpr int D = C::D, TILE = C::TILE, CH = C::CH;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  if (base - raw + C::LAYOUT_BYTES > (uint32_t)C::SMEM_BYTES) {
+    // The tiles would not fit behind the aligned base: refuse (every thread
+    // takes this branch, nothing has been started yet).
+    if (threadIdx.x == 0) atomicExch(a.status, ATTN_ERR_CUDA);
+    return;
+  }
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::OFF_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * i; };
+  auto q_off = [&](int st) -> uint32_t { return base + C::OFF_STAGE + 2 * st * TILE; };
+  auto do_off = [&](int st) -> uint32_t { return base + C::OFF_STAGE + (2 * st + 1) * TILE; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Unit order: key block slowest, so with a causal mask the blocks that see
+  // the most query blocks (the first ones) start first.
+  const int u = blockIdx.x;
+  const int kb = u / (a.Hkv * a.B);
+  const int hk = (u % (a.Hkv * a.B)) % a.Hkv;
+  const int b = (u % (a.Hkv * a.B)) / a.Hkv;
+  const int k0 = kb * C::BN;
+  int qb_start = 0;
+  if (C::CAUSAL) qb_start = max(0, (k0 - a.causal_off) / C::BM);   // first query block with a visible key
+  const int nq = max(0, a.n_qblk - qb_start);
+  const int nsteps = a.group * nq;
+  auto step_head = [&](int i) { return hk * a.group + i / nq; };
+  auto step_q0 = [&](int i) { return (qb_start + i % nq) * C::BM; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(C::B_QF + s), 1);
+      mbar_init(bar(C::B_QE + s), 1);
+    }
+    mbar_init(bar(C::B_SF), 1);
+    mbar_init(bar(C::B_DPF), 1);
+    mbar_init(bar(C::B_DQF), 1);
+    mbar_init(bar(C::B_PR), 4);
+    mbar_init(bar(C::B_DSR), 4);
+    mbar_init(bar(C::B_DQE), 4);
+    mbar_init(bar(C::B_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    if (warp == C::PRODUCER_WARP) {
+      // ---------------------------------------------------------- producer
+      if (nsteps > 0 && lane == 0) {
+        mbar_arrive_expect_tx(bar(C::B_KV), 2 * TILE);
+        for (int ch = 0; ch < C::DCH; ++ch) {
+          tma_load_4d(base + C::OFF_K + ch * CH, &tm_k, bar(C::B_KV), ch * 64, hk, k0, b);
+          tma_load_4d(base + C::OFF_V + ch * CH, &tm_v, bar(C::B_KV), ch * 64, hk, k0, b);
+        }
+      }
+      int issued = 0;
+      for (int j = 0; j < nsteps; ++j) {
+        const int st = j & 1;
+        if (!warp_wait(bar(C::B_QE + st), ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+        const int hq = step_head(j), q0 = step_q0(j);
+        float* lse_s = reinterpret_cast<float*>(base_ptr + C::OFF_ROWS + st * 1024);
+        float* dr_s = lse_s + 128;
+        const size_t rbase = ((size_t)b * a.Hq + hq) * a.Nq;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int c = 4 * lane + r, row = q0 + c;
+          float l2 = INFINITY, d = 0.f;   // rows past Nq: p = 2^-inf = 0
+          if (row < a.Nq) {
+            const float l = a.lse[rbase + row];
+            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;   // a row that saw no key keeps p = 0
+            d = a.drow[rbase + row];
+          }
+          lse_s[c] = l2;
+          dr_s[c] = d;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(C::B_QF + st), 2 * TILE);
+          for (int ch = 0; ch < C::DCH; ++ch) {
+            tma_load_4d(q_off(st) + ch * CH, &tm_q, bar(C::B_QF + st), ch * 64, hq, q0, b);
+            tma_load_4d(do_off(st) + ch * CH, &tm_do, bar(C::B_QF + st), ch * 64, hq, q0, b);
+          }
+        }
+        __syncwarp();
+        ++issued;
+      }
+      // Drain: every issued copy must land before shared memory is released.
+      if (lane == 0) {
+        for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait_drain(bar(C::B_QF + (j & 1)), (j >> 1) & 1);
+        if (nsteps > 0) mbar_wait_drain(bar(C::B_KV), 0);
+      }
+      __syncwarp();
+    } else if (warp == C::MMA_WARP) {
+      // ---------------------------------------------------------- MMA issuer
+      const bool leader = elect_one();
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, C::BM, false);     // S^T, dP^T: A, B K-major
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, true);          // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t idesc_q = idesc_bf16_f32_amn(128, D, true);      // dQ: A, B MN-major
+      bool ok = nsteps > 0 && warp_wait(bar(C::B_KV), 0, abort_flag, a.status);
+
+      // S^T_i = K Q_i^T (region A) or dP^T_i = V dO_i^T (region B): both
+      // operands K-major, k-steps of 16 along D.
+      auto issue_kmajor = [&](uint32_t a_smem, uint32_t b_smem, uint32_t d_col, uint32_t bar_done) {
+        const uint64_t adesc = sdesc_sw128(a_smem, 16, 1024);
+        const uint64_t bdesc = sdesc_sw128(b_smem, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = ((ks >> 2) * CH + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + d_col, adesc + off, bdesc + off, idesc_s, ks > 0, leader);
+        }
+        mma_commit(bar_done, leader);
+      };
+      auto wait_stage = [&](int i) -> bool {
+        if (!warp_wait(bar(C::B_QF + (i & 1)), (i >> 1) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        return true;
+      };
+
+      if (ok) ok = wait_stage(0);
+      if (ok) {
+        issue_kmajor(base + C::OFF_K, q_off(0), C::A_COL, bar(C::B_SF));
+        issue_kmajor(base + C::OFF_V, do_off(0), C::B_COL, bar(C::B_DPF));
+        __syncwarp();
+      }
+      for (int i = 0; ok && i < nsteps; ++i) {
+        const int st = i & 1;
+        if (!warp_wait(bar(C::B_PR), i & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        {   // dV += P^T dO: A = P^T (TMEM, bf16), B = dO tile read MN-major
+          const uint64_t bdesc = sdesc_sw128(do_off(st), CH, 1024);
+#pragma unroll
+          for (int ks = 0; ks < C::BM / 16; ++ks)
+            mma_ts(tmem + C::DV_COL, tmem + C::A_COL + ks * 8, bdesc + ks * 128, idesc_g, (i > 0 || ks > 0) ? 1u : 0u,
+                   leader);
+        }
+        if (i + 1 < nsteps) {
+          if (!wait_stage(i + 1)) { ok = false; break; }
+          issue_kmajor(base + C::OFF_K, q_off(st ^ 1), C::A_COL, bar(C::B_SF));
+        }
+        __syncwarp();
+        if (!warp_wait(bar(C::B_DSR), i & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        {   // dK += dS^T Q: A = dS^T (TMEM, bf16), B = Q tile read MN-major
+          const uint64_t bdesc = sdesc_sw128(q_off(st), CH, 1024);
+#pragma unroll
+          for (int ks = 0; ks < C::BM / 16; ++ks)
+            mma_ts(tmem + C::DK_COL, tmem + C::B_COL + ks * 8, bdesc + ks * 128, idesc_g, (i > 0 || ks > 0) ? 1u : 0u,
+                   leader);
+        }
+        {   // dQ = dS K: A = dS (shared memory, MN-major), B = K tile read MN-major
+          const uint64_t adesc = sdesc_sw128(base + C::OFF_DS, 128 * 128, 1024);
+          const uint64_t bdesc = sdesc_sw128(base + C::OFF_K, CH, 1024);
+#pragma unroll
+          for (int ks = 0; ks < C::BN / 16; ++ks)
+            mma_ss(tmem + C::B_COL, adesc + ks * 128, bdesc + ks * 128, idesc_q, ks > 0 ? 1u : 0u, leader);
+        }
+        mma_commit(bar(C::B_DQF), leader);
+        mma_commit(bar(C::B_QE + st), leader);
+        __syncwarp();
+        if (i + 1 < nsteps) {
+          if (!warp_wait(bar(C::B_DQE), i & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_kmajor(base + C::OFF_V, do_off(st ^ 1), C::B_COL, bar(C::B_DPF));
+          __syncwarp();
+        }
+      }
+      // Drain: no MMA may still run when TMEM is released (nothing was
+      // issued when the CTA has no step).
+      if (nsteps > 0) {
+        mma_commit(bar(C::B_DONE), leader);
+        __syncwarp();
+        mbar_wait_drain(bar(C::B_DONE), 0);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ WG0: P and dS
+    const int kr = warp * 32 + lane;      // key row in the block = TMEM lane
+    const int kk = k0 + kr;
+    const bool row_valid = kk < a.Nk;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const uint32_t tA = tmem + lane_off + C::A_COL;
+    const uint32_t tB = tmem + lane_off + C::B_COL;
+    const float sl2 = a.scale_log2;
+    for (int i = 0; i < nsteps; ++i) {
+      const int st = i & 1, q0 = step_q0(i);
+      // The stage's LSE / Drow values were stored by the producer before it
+      // arrived on the stage barrier.
+      if (!warp_wait(bar(C::B_QF + st), (i >> 1) & 1, abort_flag, a.status)) break;
+      if (!warp_wait(bar(C::B_SF), i & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint32_t rows_s = base + C::OFF_ROWS + st * 1024;
+      // P^T row, rounded to bf16 once: the same values feed the dV product
+      // and dS = P (dP - Drow) below.
+      uint32_t pk[64];
+      // Causal: key kk is visible to query q0 + c iff kk <= q0 + c + causal_off.
+      const int cmin = row_valid ? (C::CAUSAL ? kk - a.causal_off - q0 : 0) : 128;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t s[64];
+        tmem_ld64_sync(tA + half * 64, s);
+#pragma unroll
+        for (int j = 0; j < 64; j += 4) {
+          const int c = half * 64 + j;
+          uint32_t l0, l1, l2, l3;
+          ld_shared_v4(rows_s + c * 4, l0, l1, l2, l3);
+          const float p0 = ex2(fmaf(__uint_as_float(s[j + 0]), sl2, -__uint_as_float(l0)));
+          const float p1 = ex2(fmaf(__uint_as_float(s[j + 1]), sl2, -__uint_as_float(l1)));
+          const float p2 = ex2(fmaf(__uint_as_float(s[j + 2]), sl2, -__uint_as_float(l2)));
+          const float p3 = ex2(fmaf(__uint_as_float(s[j + 3]), sl2, -__uint_as_float(l3)));
+          pk[c / 2] = pack_bf16x2(p0, p1);
+          pk[c / 2 + 1] = pack_bf16x2(p2, p3);
+        }
+      }
+      if (cmin > 0) {
+        // masked columns c < cmin: clear both halves of a pair, or only its
+        // low half (column 2j) when the boundary falls inside the pair
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const uint32_t keep = (2 * j + 1 < cmin) ? 0u : (2 * j < cmin ? 0xffff0000u : 0xffffffffu);
+          pk[j] &= keep;
+        }
+      }
+      tmem_st32(tA, pk);
+      tmem_st32(tA + 32, pk + 32);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PR));
+
+      if (!warp_wait(bar(C::B_DPF), i & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint32_t ds_row = base + C::OFF_DS + kr * 128;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t dp[32];
+        tmem_ld32_sync(tB + h * 32, dp);
+        uint32_t dk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          uint32_t d0, d1, d2, d3;
+          ld_shared_v4(rows_s + 512 + (h * 32 + c) * 4, d0, d1, d2, d3);
+          const uint32_t pa = pk[(h * 32 + c) / 2], pb = pk[(h * 32 + c) / 2 + 1];
+          const float x0 = __uint_as_float(pa << 16) * (__uint_as_float(dp[c + 0]) - __uint_as_float(d0));
+          const float x1 = __uint_as_float(pa & 0xffff0000u) * (__uint_as_float(dp[c + 1]) - __uint_as_float(d1));
+          const float x2 = __uint_as_float(pb << 16) * (__uint_as_float(dp[c + 2]) - __uint_as_float(d2));
+          const float x3 = __uint_as_float(pb & 0xffff0000u) * (__uint_as_float(dp[c + 3]) - __uint_as_float(d3));
+          dk[c / 2] = pack_bf16x2(x0, x1);
+          dk[c / 2 + 1] = pack_bf16x2(x2, x3);
+        }
+        // dS^T row for dK (TMEM columns [16h, 16h+16): dP^T columns already read)
+        tmem_st16(tB + h * 16, dk);
+        // dS for dQ: A operand MN-major, 128-byte swizzle.  Atom h/2 holds
+        // queries 64(h/2) .. +63; this thread's key row is one 128-byte row
+        // of it, whose 16-byte units are permuted by (key row & 7).
+        const uint32_t atom = ds_row + (h >> 1) * (128 * 128);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t unit = uint32_t((h & 1) * 4 + v) ^ uint32_t(kr & 7);
+          st_shared_v4(atom + unit * 16, dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_DSR));
+    }
+  } else {
+    // ------------------------------------------------------------ WG1: dQ drain, dK / dV out
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;           // TMEM lane: query row of dQ, key row of dK / dV
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const uint32_t tB = tmem + lane_off + C::B_COL;
+    bool ok = true;
+    for (int i = 0; i < nsteps; ++i) {
+      const int hq = step_head(i), q = step_q0(i) + r;
+      if (!warp_wait(bar(C::B_DQF), i & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      float* dst = a.dq_acc + (((size_t)b * a.Nq + q) * a.Hq + hq) * D;
+#pragma unroll 1
+      for (int h = 0; h < D / 32; ++h) {
+        uint32_t v[32];
+        tmem_ld32_sync(tB + h * 32, v);
+        if (q < a.Nq) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            atomicAdd(reinterpret_cast<float4*>(dst + h * 32 + 4 * j),
+                      make_float4(__uint_as_float(v[4 * j]) * a.scale, __uint_as_float(v[4 * j + 1]) * a.scale,
+                                  __uint_as_float(v[4 * j + 2]) * a.scale, __uint_as_float(v[4 * j + 3]) * a.scale));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_DQE));
+    }
+    if (ok && nsteps > 0) {
+      ok = warp_wait(bar(C::B_DONE), 0, abort_flag, a.status);
+      tc_fence_after();
+    }
+    const int kk = k0 + r;
+    // Warp-uniform: the TMEM loads below are warp-collective (.sync.aligned),
+    // so every lane runs them and only the stores depend on the lane's key row.
+    const bool write = __all_sync(0xffffffffu, ok && !*abort_flag);
+    if (write) {
+      const size_t row = (((size_t)b * a.Nk + kk) * a.Hkv + hk) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* out = (which == 0 ? a.dv : a.dk) + row;
+        const float mul = which == 0 ? 1.f : a.scale;
+        const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
+#pragma unroll 1
+        for (int h = 0; h < D / 32; ++h) {
+          uint32_t v[32];
+          if (nsteps > 0) {
+            tmem_ld32_sync(tmem + lane_off + col + h * 32, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * mul, __uint_as_float(v[2 * j + 1]) * mul);
+          if (kk < a.Nk) {
+            uint4* o4 = reinterpret_cast<uint4*>(out + h * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Drow[b, h, i] = sum_d dO[b, i, h, d] * O[b, i, h, d] in fp32, one warp per
+// (b, i, h) row; the same warp zeroes that row of the fp32 dQ accumulator.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       float* __restrict__ drow, float* __restrict__ dq_acc,
+                                                       int Nq, int Hq, long long rows) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = D / 32;   // 2 or 4 elements per lane
+  const __nv_bfloat16* op = o + row * D + lane * PER;
+  const __nv_bfloat16* dp = dout + row * D + lane * PER;
+  float acc = 0.f;
+  if constexpr (PER == 4) {
+    const uint2 ov = *reinterpret_cast<const uint2*>(op);
+    const uint2 dv = *reinterpret_cast<const uint2*>(dp);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float2 of = __bfloat1622float2(o2[j]), df = __bfloat1622float2(d2[j]);
+      acc = fmaf(of.x, df.x, acc);
+      acc = fmaf(of.y, df.y, acc);
+    }
+  } else {
+    const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(op));
+    const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dp));
+    acc = fmaf(of.x, df.x, of.y * df.y);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  // row = (b * Nq + i) * Hq + h
+  const long long h = row % Hq, bi = row / Hq, i = bi % Nq, bb = bi / Nq;
+  if (lane == 0) drow[(bb * Hq + h) * Nq + i] = acc;
+  float* z = dq_acc + row * D + lane * PER;
+  if constexpr (PER == 4) *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
+  else *reinterpret_cast<float2*>(z) = make_float2(0.f, 0.f);
+}
+
+// dQ (bf16) from the fp32 accumulator, 8 elements per thread and step.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                     long long n8) {
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
+    const float4 a0 = reinterpret_cast<const float4*>(acc)[2 * t];
+    const float4 a1 = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+    reinterpret_cast<uint4*>(dq)[t] = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+                                                 pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+  }
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t workspace_bytes(int B, int Hq, int Nq, int D) {
+  const size_t n = (size_t)B * Nq * Hq;
+  return align256(n * D * 4) + align256(n * 4);
+}
+
+template <int D, bool CAUSAL>
+int launch(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, void* workspace,
+           cudaStream_t stream) {
+  using C = Cfg<D, CAUSAL>;
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* drow = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)B * Nq * Hq * D * 4));
+  const long long rows = (long long)B * Nq * Hq;
+  if (rows > 0) {
+    bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), drow, dq_acc, Nq, Hq, rows);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (Nk > 0) {
+    static int attr_done = 0;
+    const void* kfn = reinterpret_cast<const void*>(&attn_bwd_kernel<C>);
+    if (int rc = ensure_smem_attr(kfn, C::SMEM_BYTES, &attr_done)) return rc;
+    CUtensorMap tq, tk, tv, tdo;
+    const uint64_t es = 2;
+    const uint32_t box[4] = {64, 1, 128, 1};
+    {
+      // With Nq == 0 no query block is ever loaded: describe a 1-row tensor at k.
+      const uint64_t nq = Nq > 0 ? (uint64_t)Nq : 1;
+      const void* qb = Nq > 0 ? q : k;
+      const void* db = Nq > 0 ? dout : k;
+      const uint64_t hq = Nq > 0 ? (uint64_t)Hq : (uint64_t)Hkv;
+      const uint64_t dims[4] = {(uint64_t)D, hq, nq, Nq > 0 ? (uint64_t)B : 1};
+      const uint64_t strides[3] = {D * es, hq * D * es, nq * hq * D * es};
+      if (!encode_bf16_4d(&tq, qb, dims, strides, box)) return ATTN_ERR_CUDA;
+      if (!encode_bf16_4d(&tdo, db, dims, strides, box)) return ATTN_ERR_CUDA;
+    }
+    {
+      const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Nk, (uint64_t)B};
+      const uint64_t strides[3] = {D * es, (uint64_t)Hkv * D * es, (uint64_t)Nk * Hkv * D * es};
+      if (!encode_bf16_4d(&tk, k, dims, strides, box)) return ATTN_ERR_CUDA;
+      if (!encode_bf16_4d(&tv, v, dims, strides, box)) return ATTN_ERR_CUDA;
+    }
+    Args a;
+    a.lse = lse;
+    a.drow = drow;
+    a.dq_acc = dq_acc;
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.status = status;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.group = Hq / Hkv;
+    a.n_qblk = (Nq + C::BM - 1) / C::BM;
+    a.n_kblk = (Nk + C::BN - 1) / C::BN;
+    a.causal_off = Nk - Nq;
+    a.scale = scale;
+    a.scale_log2 = scale * kLog2e;
+    const long long units = (long long)a.n_kblk * Hkv * B;
+    if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    attn_bwd_kernel<C><<<(unsigned)units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (rows > 0) {
+    const long long n8 = rows * D / 8;
+    const int sms = current_sm_count();
+    const long long want = (n8 + 255) / 256;
+    const unsigned grid = (unsigned)(want < (long long)sms * 8 ? want : (long long)sms * 8);
+    bwd_dq_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // namespace bwd
+}  // namespace ea
+
+extern "C" size_t attn_bwd_workspace_size(int B, int Hq, int Nq, int D) {
+  if (B < 1 || Hq < 1 || Nq < 0 || (D != 64 && D != 128)) return 0;
+  return ea::bwd::workspace_bytes(B, Hq, Nq, D);
+}
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                        int D, int Dv, int causal, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  using namespace ea;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (Nq > 0 && (!q || !o || !dout || !lse || !dq)) return ATTN_ERR_INVALID_ARG;
+  if (Nk > 0 && (!k || !v || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != Dv) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((uint64_t)B * Nq * Hq * D * 4 >= (1ull << 40) || (uint64_t)B * Nk * Hkv * D * 2 >= (1ull << 40))
+    return ATTN_ERR_UNSUPPORTED;
+  if (Nq == 0 && Nk == 0) return ATTN_OK;
+  const size_t need = bwd::workspace_bytes(B, Hq, Nq, D);
+  if (Nq > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return ATTN_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool c = causal != 0;
+  if (D == 64)
+    return c ? bwd::launch<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, workspace, s)
+             : bwd::launch<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, workspace, s);
+  return c ? bwd::launch<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, workspace, s)
+           : bwd::launch<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, workspace, s);
+}

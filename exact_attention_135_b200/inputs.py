@@ -120,6 +120,20 @@ def prefill_config_inputs(cfg: PrefillConfig):
     return prefill_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nk, cfg.D, cfg.Dv, cfg.seed, cfg.q_mult)
 
 
+def bwd_inputs(B, Hq, Hkv, Nq, Nk, D, seed, q_mult=1.0):
+    """Backward-pass inputs: Q, K, V exactly as prefill_inputs draws them for
+    the same seed, plus the upstream gradient dO [B,Nq,Hq,D] ~ N(0,1) in bf16
+    from a second generator seeded seed + 7919."""
+    q, k, v = prefill_inputs(B, Hq, Hkv, Nq, Nk, D, D, seed, q_mult)
+    gen = torch.Generator(device="cpu").manual_seed(int(seed) + 7919)
+    do = _randn_bf16(gen, (B, Nq, Hq, D))
+    return q, k, v, do
+
+
+def bwd_config_inputs(cfg: PrefillConfig):
+    return bwd_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nk, cfg.D, cfg.seed, cfg.q_mult)
+
+
 @dataclass
 class PagedCache:
     q: torch.Tensor              # [B, 1, Hq, Dk] bf16

@@ -84,6 +84,47 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              int Nk, int D, int Dv, int causal, float scale, void* stream);
 
 /*
+ * attn_bwd_workspace_size: bytes of device workspace that attn_bwd needs for
+ * B x Nq query rows of Hq heads of width D (an fp32 dQ accumulator plus one
+ * fp32 value per query row).  0 for an unsupported D.  The caller allocates
+ * it, 256-byte aligned.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Nq, int D);
+
+/*
+ * attn_bwd: gradients of attn_fwd with respect to q, k and v, with S and P
+ * recomputed block by block from q, k and the forward's LSE ("Flash
+ * Attention" wiki page, section "구조화된 지식 (Synthesized Content)", item
+ * "Recomputation (재계산)": the backward pass recomputes what it needs
+ * instead of storing N x N matrices).  For an upstream gradient dout = dL/dO:
+ *
+ *   P = exp(scale * q k^T - lse) (0 where masked), dv = P^T dout,
+ *   dP = dout v^T, dS = P * (dP - rowsum(dout * o)),
+ *   dq = scale * dS k, dk = scale * dS^T q
+ *
+ * with dk and dv summed over the query heads that share a KV head.
+ *
+ *   q, o, dout  [B, Nq, Hq, D] bf16     k, v [B, Nk, Hkv, D] bf16
+ *   lse         [B, Hq, Nq] fp32, as written by attn_fwd for the same inputs
+ *   dq          [B, Nq, Hq, D] bf16 (written)
+ *   dk, dv      [B, Nk, Hkv, D] bf16 (written)
+ *   workspace   at least attn_bwd_workspace_size(B, Hq, Nq, D) bytes; content
+ *               on entry irrelevant, undefined on return
+ *
+ * causal, scale, the head grouping and the mask alignment are those of
+ * attn_fwd.  Supported: D == Dv in {64, 128}; Hq % Hkv == 0; scale finite and
+ * > 0; tensors 16-byte aligned, lse 4-byte aligned.  Accumulation is fp32; P
+ * and dS are rounded to bf16 before their products; outputs are rounded to
+ * bf16 once.  dk and dv are deterministic run to run; dq is accumulated with
+ * fp32 atomic adds (one per key block), so its last bits may vary from run
+ * to run.  Returns ATTN_ERR_WORKSPACE if the workspace is missing, too small
+ * or misaligned.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int D, int Dv, int causal,
+             float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_paged_workspace_size: bytes of device workspace that
  * attn_decode_paged needs for a batch of B sequences with Hq heads of width
  * Dv on the current device.  The caller allocates it (any alignment >= 256 B).

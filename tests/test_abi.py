@@ -109,3 +109,26 @@ def test_mtp_decode_argument_checks(lib):
     assert call(Hq=64) == 2
     assert call(B=1024, s_q=4) == 2          # more than 2048 query units
     assert lib.attn_decode_paged_mtp_workspace_size(1024, 4, 128, 512) == 0
+
+
+def test_bwd_argument_checks(lib):
+    def call(q=A, lse=A, dk=A, B=1, Hq=4, Hkv=2, Nq=100, Nk=100, D=128, Dv=128, scale=0.1, ws=A, wsb=1 << 30):
+        return lib.attn_bwd(q, A, A, A, A, lse, A, dk, A, B, Hq, Hkv, Nq, Nk, D, Dv, 1, scale, ws, wsb, None)
+    assert call(q=None) == 1
+    assert call(dk=None) == 1
+    assert call(lse=A + 2) == 1              # misaligned
+    assert call(Hq=6, Hkv=4) == 1            # Hq % Hkv
+    assert call(B=0) == 1
+    assert call(Nq=-1) == 1
+    assert call(scale=0.0) == 1
+    assert call(scale=float("inf")) == 1
+    assert call(D=256, Dv=256) == 2          # dK and dV do not fit TMEM next to the work tiles
+    assert call(D=128, Dv=64) == 2
+    assert call(D=96, Dv=96) == 2
+    assert call(ws=None) == 5
+    assert call(wsb=1024) == 5
+    assert call(ws=A + 16) == 5              # workspace must be 256-byte aligned
+    assert call(Nq=0, Nk=0, q=None, dk=None, ws=None, wsb=0) == 0
+    need = lib.attn_bwd_workspace_size(1, 4, 100, 128)
+    assert need >= 100 * 4 * 128 * 4 + 100 * 4 * 4
+    assert lib.attn_bwd_workspace_size(1, 4, 100, 256) == 0
