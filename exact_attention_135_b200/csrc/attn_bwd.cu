@@ -19,13 +19,16 @@
 //   attn_bwd_kernel   one CTA per (key block of 128, KV head, batch).  dK and dV
 //                     stay in TMEM while the CTA walks every query block of
 //                     every query head of the group that sees its keys; each
-//                     step's dQ contribution is added to the accumulator
+//                     step's dQ contribution is added to the accumulator by a
+//                     TMA reduce-add (at L2, coalesced whole tiles)
 //   bwd_dq_kernel     dQ accumulator -> bf16
 //
-// Roles inside attn_bwd_kernel (320 threads, 200 registers each):
-//   warps 0-3  (WG0)  one key row per thread: S^T, dP^T from TMEM, P and dS -> bf16
-//                     into TMEM (for dV, dK) and dS into shared memory (for dQ)
-//   warps 4-7  (WG1)  one query row per thread: dQ from TMEM -> fp32 atomics;
+// Roles inside attn_bwd_kernel (320 threads):
+//   warps 0-3  (WG0)  one key row per thread: S^T, dP^T from TMEM, P -> bf16 into
+//                     TMEM (for dV) and dS -> bf16 into shared memory (for dK
+//                     and dQ: the same tile is K-major for dS^T and MN-major for dS)
+//   warps 4-7  (WG1)  one query row per thread: dQ from TMEM -> shared memory
+//                     (the dS tile, free once dQ is computed) -> TMA reduce-add;
 //                     at the end dK, dV -> bf16 -> global
 //   warp 8            TMA: K, V once; a two-stage ring of (Q, dO) tiles plus the
 //                     step's LSE and Drow values
@@ -33,10 +36,10 @@
 //
 // TMEM (128 lanes x 512 fp32 columns): dV [0, D), dK [D, 2D), region A
 // [2D, 2D+128) = S^T then P^T (bf16, first 64 columns), region B
-// [2D+128, 2D+256) = dP^T then dS^T (bf16, first 64 columns) then dQ.  Issue
-// order per step i (tcgen05.mma executes in issue order, so an MMA may
-// overwrite columns an earlier one reads):
-//   dV_i (reads P^T_i) -> S^T_{i+1} (A) -> dK_i (reads dS^T_i) -> dQ_i (B)
+// [2D+128, 2D+256) = dP^T then dQ.  Issue order per step i (tcgen05.mma
+// executes in issue order, so an MMA may overwrite columns an earlier one
+// reads):
+//   dV_i (reads P^T_i) -> S^T_{i+1} (A) -> dK_i, dQ_i (read dS_i; dQ_i -> B)
 //   -> [dQ_i drained by WG1] -> dP^T_{i+1} (B)
 // so the next step's S^T is computed while WG0 still forms dS_i, and dQ's
 // drain overlaps the next step's softmax work.
@@ -57,7 +60,7 @@ struct Cfg {
   static constexpr int DCH = D / 64;               // 128-byte column chunks of a tile
   static constexpr int CH = 128 * 128;             // bytes of one chunk of a 128-row tile
   static constexpr int TILE = 128 * D * 2;         // bytes of one 128-row bf16 tile
-  static constexpr int DS_BYTES = BM * BN * 2;     // dS tile, A operand of dQ (MN-major)
+  static constexpr int DS_BYTES = BM * BN * 2;     // dS tile (A of dK K-major, A of dQ MN-major); dQ staging
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
@@ -101,7 +104,6 @@ struct Cfg {
 struct Args {
   const float* lse;      // [B, Hq, Nq] natural log
   const float* drow;     // [B, Hq, Nq]
-  float* dq_acc;         // [B, Nq, Hq, D]
   __nv_bfloat16* dk;     // [B, Nk, Hkv, D]
   __nv_bfloat16* dv;     // [B, Nk, Hkv, D]
   int* status;
@@ -115,7 +117,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const Args a) {
+                    const __grid_constant__ CUtensorMap tm_dq, const Args a) {
   constexpr int D = C::D, TILE = C::TILE, CH = C::CH;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -145,8 +147,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (C::CAUSAL) qb_start = max(0, (k0 - a.causal_off) / C::BM);   // first query block with a visible key
   const int nq = max(0, a.n_qblk - qb_start);
   const int nsteps = a.group * nq;
-  auto step_head = [&](int i) { return hk * a.group + i / nq; };
-  auto step_q0 = [&](int i) { return (qb_start + i % nq) * C::BM; };
+  // Steps walk the query blocks in order, the group's heads innermost: the
+  // CTAs resident at one time (neighbouring key blocks) then work on
+  // neighbouring query blocks, so the dQ accumulator rows they add into and
+  // the Q / dO tiles they read stay in L2.
+  auto step_head = [&](int i) { return hk * a.group + i % a.group; };
+  auto step_q0 = [&](int i) { return (qb_start + i / a.group) * C::BM; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
@@ -169,6 +175,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 0) {
     tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // ---------------------------------------------------------- MMA issuer
       const bool leader = elect_one();
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, C::BM, false);     // S^T, dP^T: A, B K-major
-      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, true);          // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, true);          // dV: A in TMEM; dK: A K-major; B MN-major
       constexpr uint32_t idesc_q = idesc_bf16_f32_amn(128, D, true);      // dQ: A, B MN-major
       bool ok = nsteps > 0 && warp_wait(bar(C::B_KV), 0, abort_flag, a.status);
 
@@ -276,12 +283,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
         if (!warp_wait(bar(C::B_DSR), i & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        {   // dK += dS^T Q: A = dS^T (TMEM, bf16), B = Q tile read MN-major
+        {   // dK += dS^T Q: A = dS^T (the dS tile read K-major: key rows, queries along K),
+            // B = Q tile read MN-major
+          const uint64_t adesc = sdesc_sw128(base + C::OFF_DS, 16, 1024);
           const uint64_t bdesc = sdesc_sw128(q_off(st), CH, 1024);
 #pragma unroll
-          for (int ks = 0; ks < C::BM / 16; ++ks)
-            mma_ts(tmem + C::DK_COL, tmem + C::B_COL + ks * 8, bdesc + ks * 128, idesc_g, (i > 0 || ks > 0) ? 1u : 0u,
-                   leader);
+          for (int ks = 0; ks < C::BM / 16; ++ks) {
+            const uint32_t a_off = ((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4;
+            mma_ss(tmem + C::DK_COL, adesc + a_off, bdesc + ks * 128, idesc_g, (i > 0 || ks > 0) ? 1u : 0u, leader);
+          }
         }
         {   // dQ = dS K: A = dS (shared memory, MN-major), B = K tile read MN-major
           const uint64_t adesc = sdesc_sw128(base + C::OFF_DS, 128 * 128, 1024);
@@ -371,7 +381,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int h = 0; h < 4; ++h) {
         uint32_t dp[32];
         tmem_ld32_sync(tB + h * 32, dp);
-        uint32_t dk[16];
+        uint32_t ds[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           uint32_t d0, d1, d2, d3;
@@ -381,22 +391,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const float x1 = __uint_as_float(pa & 0xffff0000u) * (__uint_as_float(dp[c + 1]) - __uint_as_float(d1));
           const float x2 = __uint_as_float(pb << 16) * (__uint_as_float(dp[c + 2]) - __uint_as_float(d2));
           const float x3 = __uint_as_float(pb & 0xffff0000u) * (__uint_as_float(dp[c + 3]) - __uint_as_float(d3));
-          dk[c / 2] = pack_bf16x2(x0, x1);
-          dk[c / 2 + 1] = pack_bf16x2(x2, x3);
+          ds[c / 2] = pack_bf16x2(x0, x1);
+          ds[c / 2 + 1] = pack_bf16x2(x2, x3);
         }
-        // dS^T row for dK (TMEM columns [16h, 16h+16): dP^T columns already read)
-        tmem_st16(tB + h * 16, dk);
-        // dS for dQ: A operand MN-major, 128-byte swizzle.  Atom h/2 holds
-        // queries 64(h/2) .. +63; this thread's key row is one 128-byte row
-        // of it, whose 16-byte units are permuted by (key row & 7).
+        // dS tile, 128-byte swizzle: atom h/2 holds queries 64(h/2) .. +63;
+        // this thread's key row is one 128-byte row of it, whose 16-byte
+        // units are permuted by (key row & 7).  Read K-major it is dS^T
+        // (A of dK), read MN-major it is dS (A of dQ).
         const uint32_t atom = ds_row + (h >> 1) * (128 * 128);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const uint32_t unit = uint32_t((h & 1) * 4 + v) ^ uint32_t(kr & 7);
-          st_shared_v4(atom + unit * 16, dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          st_shared_v4(atom + unit * 16, ds[4 * v], ds[4 * v + 1], ds[4 * v + 2], ds[4 * v + 3]);
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -408,28 +416,50 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int r = wq * 32 + lane;           // TMEM lane: query row of dQ, key row of dK / dV
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t tB = tmem + lane_off + C::B_COL;
+    const uint32_t stage_s = base + C::OFF_DS;   // dS tile: free once dQ_i is in TMEM
+    const bool issuer = (wq == 0 && lane == 0);
     bool ok = true;
     for (int i = 0; i < nsteps; ++i) {
-      const int hq = step_head(i), q = step_q0(i) + r;
-      if (!warp_wait(bar(C::B_DQF), i & 1, abort_flag, a.status)) { ok = false; break; }
+      const int hq = step_head(i), q0 = step_q0(i);
+      // all four warps take the same decision, so none is left at a named barrier
+      ok = named_bar_and(1, 128, warp_wait(bar(C::B_DQF), i & 1, abort_flag, a.status));
+      if (!ok) break;
       tc_fence_after();
-      float* dst = a.dq_acc + (((size_t)b * a.Nq + q) * a.Hq + hq) * D;
+      // dQ_i in rounds of 64 columns: two 32-column fp32 boxes (128 rows x
+      // 128 bytes, 128-byte swizzle) staged in the dS tile, then added into
+      // the accumulator by the TMA unit (rows past Nq are clipped).
 #pragma unroll 1
-      for (int h = 0; h < D / 32; ++h) {
-        uint32_t v[32];
-        tmem_ld32_sync(tB + h * 32, v);
-        if (q < a.Nq) {
+      for (int rnd = 0; rnd < D / 64; ++rnd) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            atomicAdd(reinterpret_cast<float4*>(dst + h * 32 + 4 * j),
-                      make_float4(__uint_as_float(v[4 * j]) * a.scale, __uint_as_float(v[4 * j + 1]) * a.scale,
-                                  __uint_as_float(v[4 * j + 2]) * a.scale, __uint_as_float(v[4 * j + 3]) * a.scale));
+        for (int bx = 0; bx < 2; ++bx) {
+          uint32_t v[32];
+          tmem_ld32_sync(tB + rnd * 64 + bx * 32, v);
+          const uint32_t row_s = stage_s + bx * (128 * 128) + r * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t unit = uint32_t(u) ^ uint32_t(r & 7);
+            st_shared_v4(row_s + unit * 16, __float_as_uint(__uint_as_float(v[4 * u]) * a.scale),
+                         __float_as_uint(__uint_as_float(v[4 * u + 1]) * a.scale),
+                         __float_as_uint(__uint_as_float(v[4 * u + 2]) * a.scale),
+                         __float_as_uint(__uint_as_float(v[4 * u + 3]) * a.scale));
+          }
         }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+            tma_reduce_add_4d(&tm_dq, stage_s + bx * (128 * 128), rnd * 64 + bx * 32, hq, q0, b);
+          tma_store_commit();
+          tma_store_wait_read();   // the staging tile may be overwritten again
+        }
+        named_bar_sync(1, 128);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_DQE));
     }
+    if (issuer) tma_store_wait_all();   // every reduce has landed before the CTA ends
     if (ok && nsteps > 0) {
       ok = warp_wait(bar(C::B_DONE), 0, abort_flag, a.status);
       tc_fence_after();
@@ -574,10 +604,21 @@ int launch(const void* q, const void* k, const void* v, const void* o, const voi
       if (!encode_bf16_4d(&tk, k, dims, strides, box)) return ATTN_ERR_CUDA;
       if (!encode_bf16_4d(&tv, v, dims, strides, box)) return ATTN_ERR_CUDA;
     }
+    CUtensorMap tdq;
+    {
+      // fp32 dQ accumulator [B, Nq, Hq, D], 32-column boxes (128 bytes);
+      // with Nq == 0 nothing is ever added: describe one row at k.
+      const uint64_t nq = Nq > 0 ? (uint64_t)Nq : 1;
+      const void* base_dq = Nq > 0 ? static_cast<const void*>(dq_acc) : k;
+      const uint64_t hq = Nq > 0 ? (uint64_t)Hq : 1;
+      const uint64_t dq_dims[4] = {Nq > 0 ? (uint64_t)D : 32, hq, nq, Nq > 0 ? (uint64_t)B : 1};
+      const uint64_t dq_strides[3] = {dq_dims[0] * 4, hq * dq_dims[0] * 4, nq * hq * dq_dims[0] * 4};
+      const uint32_t dq_box[4] = {32, 1, 128, 1};
+      if (!encode_f32_4d(&tdq, base_dq, dq_dims, dq_strides, dq_box)) return ATTN_ERR_CUDA;
+    }
     Args a;
     a.lse = lse;
     a.drow = drow;
-    a.dq_acc = dq_acc;
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
     a.status = status;
@@ -594,7 +635,7 @@ int launch(const void* q, const void* k, const void* v, const void* o, const voi
     a.scale_log2 = scale * kLog2e;
     const long long units = (long long)a.n_kblk * Hkv * B;
     if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    attn_bwd_kernel<C><<<(unsigned)units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    attn_bwd_kernel<C><<<(unsigned)units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, a);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (rows > 0) {

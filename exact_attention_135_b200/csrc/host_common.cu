@@ -31,8 +31,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                 const uint32_t* box) {
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
+                  const uint64_t* strides, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t d[5], s[4];
@@ -43,7 +43,7 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
     es[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) s[i] = strides[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, bx, es,
+  CUresult r = fn(map, dtype, rank, const_cast<void*>(base), d, s, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -77,17 +77,22 @@ int current_sm_count() {
 
 bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                     const uint32_t box[4]) {
-  return encode_bf16(map, base, 4, dims, strides, box);
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, strides, box);
+}
+
+bool encode_f32_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                   const uint32_t box[4]) {
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 4, dims, strides, box);
 }
 
 bool encode_bf16_2d(CUtensorMap* map, const void* base, const uint64_t dims[2], const uint64_t strides[1],
                     const uint32_t box[2]) {
-  return encode_bf16(map, base, 2, dims, strides, box);
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, strides, box);
 }
 
 bool encode_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
                     const uint32_t box[3]) {
-  return encode_bf16(map, base, 3, dims, strides, box);
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, strides, box);
 }
 
 int ensure_smem_attr(const void* kernel, int bytes, int* done_mask) {

@@ -23,6 +23,10 @@ int* device_status_ptr();
 bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                     const uint32_t box[4]);
 
+// The same for fp32 elements (box[0] * 4 bytes must be <= 128).
+bool encode_f32_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                   const uint32_t box[4]);
+
 // Encode a 2-D bf16 tile map with 128-byte swizzle (stride of dim 1).
 bool encode_bf16_2d(CUtensorMap* map, const void* base, const uint64_t dims[2], const uint64_t strides[1],
                     const uint32_t box[2]);
