@@ -56,7 +56,7 @@ NCU_TRAFFIC_BYTES = {
     "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
     "decode": 349649664 + 16860928,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
-    "bwd": None,                        # attn_bwd_kernel<D=128, causal>: not captured yet
+    "bwd": 2549769216 + 1224851200,     # attn_bwd_kernel<D=128, causal>, same workload (backward)
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.
