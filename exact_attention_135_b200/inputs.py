@@ -120,6 +120,34 @@ def prefill_config_inputs(cfg: PrefillConfig):
     return prefill_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nk, cfg.D, cfg.Dv, cfg.seed, cfg.q_mult)
 
 
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor FP8 (E4M3) encoding of an fp32 tensor for the FP8 forward.
+
+    descale = max|x| / 448, rounded to fp32 (the value both the kernel and
+    the oracle then use); the bytes are x / descale rounded to nearest even
+    by torch's float8_e4m3fn cast, returned as uint8.  Returns (bytes, descale).
+    """
+    amax = float(x.abs().max()) if x.numel() else 0.0
+    descale = float(torch.tensor(amax / E4M3_MAX if amax > 0 else 1.0, dtype=torch.float32))
+    q = (x / descale).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8), descale
+
+
+def fp8_prefill_inputs(B, Hq, Hkv, Nq, Nk, D, seed, q_mult=1.0):
+    """FP8 forward inputs: Q, K, V drawn as prefill_inputs draws them (the same
+    generator stream, kept in fp32 instead of rounded to bf16), then each
+    encoded per tensor by quantize_e4m3.  Returns (q8, k8, v8, (dq, dk, dv))."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = torch.randn(B, Nq, Hq, D, generator=gen, dtype=torch.float32) * q_mult
+    k = torch.randn(B, Nk, Hkv, D, generator=gen, dtype=torch.float32)
+    v = torch.randn(B, Nk, Hkv, D, generator=gen, dtype=torch.float32)
+    (q8, dq), (k8, dk), (v8, dv) = quantize_e4m3(q), quantize_e4m3(k), quantize_e4m3(v)
+    return q8, k8, v8, (dq, dk, dv)
+
+
 def bwd_inputs(B, Hq, Hkv, Nq, Nk, D, seed, q_mult=1.0):
     """Backward-pass inputs: Q, K, V exactly as prefill_inputs draws them for
     the same seed, plus the upstream gradient dO [B,Nq,Hq,D] ~ N(0,1) in bf16

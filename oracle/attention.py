@@ -29,6 +29,11 @@ What it computes is the plain definition the fused kernels must reach exactly
   of query heads reads its own group-expanded cache.  Here that is a paged
   cache of separate K and V rows per (token, KV head); query head h reads KV
   head h // (Hq / Hkv), as in the dense oracle.
+* "FlashAttention (KO)", section "FlashAttention-3 (2024)": FP8 inputs.  The
+  page names no format; ``e4m3_decode`` follows the OCP 8-bit floating-point
+  definition of E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits,
+  subnormals at exponent field 0, no infinities, S.1111.111 is NaN), and
+  ``attention_fp8`` is exact attention on the values the bytes represent.
 * "Flash Attention" wiki page, section "구조화된 지식 (Synthesized Content)",
   item "Recomputation (재계산)": the backward pass recomputes the intermediate
   matrices instead of storing them.  ``attention_bwd`` writes out the plain
@@ -46,6 +51,8 @@ values (tests/golden/), closed forms, invariants, a pure-Python brute force
 and torch's fp64 scaled_dot_product_attention; tests/test_oracle_gqa.py and
 tests/test_oracle_mtp.py pin the GQA-path and multi-token decode functions
 with brute forces, closed forms, invariances and planted mistakes;
+tests/test_oracle_fp8.py pins the E4M3 decoding against torch's float8_e4m3fn,
+hand-derived codes and planted mistakes;
 tests/test_oracle_bwd.py pins the gradients with central finite differences
 of the forward function, torch fp64 autograd, closed forms, the zero sum of
 the dK rows and planted mistakes.
@@ -55,7 +62,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention", "attention_bwd", "decode_paged", "decode_paged_mtp", "decode_paged_gqa", "gather_pages"]
+__all__ = ["attention", "attention_bwd", "attention_fp8", "decode_paged", "decode_paged_mtp", "decode_paged_gqa",
+           "e4m3_decode", "gather_pages"]
 
 
 def _rows_softmax_weighted(S: np.ndarray, V: np.ndarray):
@@ -306,3 +314,35 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float, q_rows=None, k_rows=N
                     if sel:
                         dQ[b, [q_pos[int(rows[i])] for i in sel], hq, :] = scale * (dS[sel] @ Kmat)
     return dQ, dK, dV
+
+
+def e4m3_decode(codes):
+    """Values of OCP FP8 E4M3 bytes, in fp64 (NaN for the two NaN codes).
+
+    Bit layout s eeee mmm: exponent field e in 1..15 gives
+    (-1)^s * 2^(e - 7) * (1 + m/8); e = 0 gives the subnormals
+    (-1)^s * 2^-6 * (m/8); e = 15 with m = 7 is NaN (the format has no
+    infinities, so 0x7E = 448 is the largest finite value).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + m / 8.0, e - 7)
+    sub = sign * np.ldexp(m / 8.0, -6)
+    out = np.where(e == 0, sub, normal)
+    return np.where((e == 15) & (m == 7), np.nan, out)
+
+
+def attention_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float, causal: bool, scale: float,
+                  q_rows=None):
+    """Exact attention on FP8 inputs: the definition of ``attention`` applied
+    to the represented values descale * e4m3(byte), in fp64.
+
+    q8 [B, Nq, Hq, D], k8 [B, Nk, Hkv, D], v8 [B, Nk, Hkv, D]: E4M3 bytes.
+    Returns O and LSE as ``attention`` does.
+    """
+    q = q_descale * e4m3_decode(q8)
+    k = k_descale * e4m3_decode(k8)
+    v = v_descale * e4m3_decode(v8)
+    return attention(q, k, v, causal, scale, q_rows=q_rows)
