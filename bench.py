@@ -14,6 +14,7 @@ already resident in device memory:
     the same length mix);
   * mtp:     attn_decode_paged_mtp, the MLA decode with two query tokens per
     sequence;
+  * fp8:     attn_fwd_fp8, the prefill on E4M3 inputs (same shape);
   * bwd:     attn_bwd (gradients of the prefill) on the long-context workload.
 The headline metric is prefill TFLOP/s (4*Nq*Nk*D per head, halved for
 causal); the decode KV-cache GB/s (bytes of the K/V rows of valid tokens
@@ -57,6 +58,7 @@ NCU_TRAFFIC_BYTES = {
     "decode": 349649664 + 16860928,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
     "bwd": 2549769216 + 1224851200,     # attn_bwd_kernel<D=128, causal>, same workload (backward)
+    "fp8": 100732160 + 92020992,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.
@@ -269,6 +271,28 @@ def gqa_part(ea, dev):
     return p
 
 
+def fp8_part(ea, dev):
+    """attn_fwd_fp8 on the long-context GQA causal shape with E4M3 inputs
+    (the same draws as the prefill workload, encoded per tensor)."""
+    cfg = inputs.PREFILL_CONFIGS[PREFILL_ID]
+    q8, k8, v8, ds = inputs.fp8_prefill_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.Nq, cfg.Nk, cfg.D, cfg.seed, cfg.q_mult)
+    host = {"q": q8.pin_memory(), "k": k8.pin_memory(), "v": v8.pin_memory()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    d["o"] = torch.empty((cfg.B, cfg.Nq, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=dev)
+    d["lse"] = torch.empty((cfg.B, cfg.Hq, cfg.Nq), dtype=torch.float32, device=dev)
+    host["o"] = torch.empty(d["o"].shape, dtype=torch.bfloat16).pin_memory()
+    host["lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
+
+    def run():
+        ea.fwd_fp8(d["q"], d["k"], d["v"], *ds, causal=cfg.causal, scale=cfg.scale, out=d["o"], lse=d["lse"])
+
+    p = Part("fp8", run, [(d[n], host[n]) for n in ("q", "k", "v")],
+             [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=1)
+    p.cfg = cfg
+    p.work = cfg.flops()
+    return p
+
+
 def bwd_part(ea, dev):
     """attn_bwd on the long-context GQA causal workload: O and LSE come from
     one forward pass at setup; dO ~ N(0,1) bf16 from its own seeded stream."""
@@ -357,6 +381,8 @@ def run_gpu(args):
         parts.append(gqa_part(ea, dev))
     if args.part in ("all", "mtp"):
         parts.append(mtp_part(ea, dev))
+    if args.part in ("all", "fp8"):
+        parts.append(fp8_part(ea, dev))
     if args.part in ("all", "bwd"):
         parts.append(bwd_part(ea, dev))
 
@@ -459,6 +485,24 @@ def run_gpu(args):
     sustained = step_ms * args.steps * 1e-3 > SUSTAINED_AFTER_S
     bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     bf16_kind = f"{peaks_kind} bf16 {'sustained' if sustained else 'burst'}"
+    fp8_obj = None
+    if "fp8" in by:
+        p = by["fp8"]
+        tf = p.work / (launch_ms["fp8"] * 1e-3) / 1e12
+        # no measured fp8 peak: the measured bf16 peak times the nominal dense fp8/bf16 ratio (4.5 / 2.25)
+        fp8_peak = 2.0 * bf16_peak
+        fp8_obj = {
+            "metric": "attention TFLOP/s (FP8 E4M3 prefill)",
+            "value": round(whole_job_rate(world, p.work, launch_ms["fp8"]) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_launch": round(launch_ms["fp8"], 4),
+            "config": {"workload": p.cfg.name + ", E4M3 inputs with per-tensor descales", "dtype": "e4m3"},
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(tf / fp8_peak, 4), "peak_kind": bf16_kind + " x 2 (nominal fp8/bf16 ratio)",
+                         "traffic": NCU_TRAFFIC_BYTES["fp8"], "kernel": "attn_fwd_kernel<D=128,causal,fp8>",
+                         "frac_of_bf16_peak": round(tf / bf16_peak, 4)},
+            "e2e": {"value": round(world * p.work / (e2e_ms["fp8"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
+        }
     bwd_obj = None
     if "bwd" in by:
         p = by["bwd"]
@@ -505,10 +549,12 @@ def run_gpu(args):
             line["gqa_decode"] = gqa_obj
         if mtp_obj:
             line["decode_mtp"] = mtp_obj
+        if fp8_obj:
+            line["fp8"] = fp8_obj
         if bwd_obj:
             line["bwd"] = bwd_obj
     else:
-        head = decode_obj or gqa_obj or mtp_obj or bwd_obj
+        head = decode_obj or gqa_obj or mtp_obj or fp8_obj or bwd_obj
         line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
         line["config"]["step"] = step_parts
         if decode_obj and gqa_obj:
@@ -611,7 +657,7 @@ def main():
     ap.add_argument("--baseline-rows", type=int, default=768,
                     help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp", "bwd"], default="all",
+    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp", "fp8", "bwd"], default="all",
                     help="time only one piece of the step (for profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()

@@ -58,6 +58,7 @@ _SIGNATURES = {
     "attn_decode_paged_mtp_workspace_size": (_sz, [_i, _i, _i, _i]),
     "attn_decode_paged_mtp": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _f, _f, _f, _vp, _vp] + [_i] * 7 + [_f, _vp]),
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _sz, _vp]),
 }
@@ -140,6 +141,39 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                                 B, Hq, Hkv, Nq, Nk, D, Dv, int(bool(causal)), float(scale),
                                 _stream_handle(q.device))
     _check(rc, "attn_fwd")
+    return out, lse
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float, k_descale: float,
+            v_descale: float, causal: bool = False, scale: float | None = None, out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None):
+    """Fused exact attention forward on e4m3 inputs.
+
+    q [B,Nq,Hq,D], k [B,Nk,Hkv,D], v [B,Nk,Hkv,D] CUDA tensors of e4m3 bytes
+    (torch.float8_e4m3fn or uint8); the represented values are descale * e4m3.
+    Returns (o [B,Nq,Hq,D] bf16, lse [B,Hq,Nq] fp32).  D must be 128.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise TypeError(f"{n} must hold e4m3 bytes (float8_e4m3fn or uint8), got {t.dtype}")
+        _need(t, n, t.dtype, 4)
+    B, Nq, Hq, D = q.shape
+    Bk, Nk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D or tuple(v.shape) != (B, Nk, Hkv, D):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Nq, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    with torch.cuda.device(q.device):
+        rc = library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_descale), float(k_descale),
+                                    float(v_descale), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nk, D,
+                                    int(bool(causal)), float(scale), _stream_handle(q.device))
+    _check(rc, "attn_fwd_fp8")
     return out, lse
 
 

@@ -29,25 +29,41 @@
 
 namespace ea {
 
-template <int D_, bool CAUSAL_, int BN_>
+template <int D_, bool CAUSAL_, int BN_, bool FP8_ = false>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr bool CAUSAL = CAUSAL_;
+  // FP8: Q, K, V are e4m3 bytes and P is rounded to e4m3 for P V (O, LSE as
+  // in the bf16 path).
+  static constexpr bool FP8 = FP8_;
+  static constexpr int ES = FP8 ? 1 : 2;             // bytes per Q/K/V element
   static constexpr int BM = 128;                     // query rows per tile = TMEM lanes
   static constexpr int NT = (D <= 128) ? 2 : 1;      // Q tiles per CTA
   static constexpr int BN = BN_;                     // keys per block
   // S buffers per tile: two whenever they fit next to O in the tile's 256
   // TMEM columns, so S of block j+1 overlaps the softmax of block j.
   static constexpr int NSL = (NT == 1 || 2 * BN + D <= 256) ? 2 : 1;
-  static constexpr int KV_TILE = BN * D * 2;
-  static constexpr int KV_BUDGET = 224 * 1024 - NT * BM * D * 2;      // shared memory left for K/V
+  static constexpr int KV_TILE = BN * D * ES;
+  // FP8 stages the bf16 O tiles in a region of their own (the e4m3 Q tile is
+  // half their size); bf16 reuses the dead Q tile.
+  static constexpr int O_STAGE_BYTES = FP8 ? NT * 128 * D * 2 : 0;
+  static constexpr int KV_BUDGET = 224 * 1024 - NT * BM * D * ES - O_STAGE_BYTES;   // shared memory left for K/V
   static constexpr int KSTAGES = (KV_BUDGET / KV_TILE + 1) / 2;      // K ring (released after S)
   static constexpr int VSTAGES = KV_BUDGET / KV_TILE - KSTAGES;      // V ring (held until P V)
-  static constexpr int DCH = D / 64;                 // 128-byte column chunks
+  static constexpr int DCH = D * ES / 128;           // 128-byte column chunks
+  static constexpr int CH_ELEMS = 128 / ES;          // elements in a 128-byte chunk row
+  static constexpr int K_MMA = 32 / ES;              // reduction depth of one MMA (32 bytes)
+  static constexpr int P_WORDS = BN * ES / 4;        // TMEM columns of one packed P row
   static constexpr int Q_CHUNK = BM * 128;           // bytes of one chunk of a Q tile
   static constexpr int KV_CHUNK = BN * 128;
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int Q_BYTES = BM * D * ES;
+  static constexpr int KV_BYTES = BN * D * ES;
+  // Lazy rescale: O is rescaled only when a row max grows by more than 2^THR.
+  // FP8 also measures p from 2^SHIFT below the running max, so that p lies in
+  // (0, 2^(THR + SHIFT)] = (0, 256]: inside e4m3's range (max 448) and mostly
+  // above its smallest normal (2^-6).
+  static constexpr float RESCALE_THR = FP8 ? 4.0f : 8.0f;
+  static constexpr float P_SHIFT = FP8 ? 4.0f : 0.0f;
   static constexpr int SOFTMAX_WARPS = 4 * NT;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // Q and K loads
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
@@ -85,7 +101,8 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VSTAGES * KV_BYTES;
+  static constexpr int OFF_OST = OFF_V + VSTAGES * KV_BYTES;   // FP8 only: bf16 O staging
+  static constexpr int OFF_BAR = OFF_OST + O_STAGE_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -98,10 +115,10 @@ struct FwdArgs {
   float* lse;
   int* status;
   int Hq, Nq, Nk, group, n_qblk, causal_off;
-  float scale_log2;
+  float scale_log2;   // scale * log2(e) (FP8: times the Q and K descales)
+  float o_mul;        // 1 (FP8: the V descale)
 };
 
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when the max grows by > 2^8
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <class C>
@@ -196,8 +213,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mbar_arrive_expect_tx(bar(C::B_QF + t), C::Q_BYTES);
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_4d(base + C::OFF_Q + t * C::Q_BYTES + ch * C::Q_CHUNK, &tm_q, bar(C::B_QF + t), ch * 64, hq,
-                        r0, b);
+            tma_load_4d(base + C::OFF_Q + t * C::Q_BYTES + ch * C::Q_CHUNK, &tm_q, bar(C::B_QF + t),
+                        ch * C::CH_ELEMS, hq, r0, b);
         }
       }
       int k_issued = 0;
@@ -207,8 +224,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_4d(base + C::OFF_K + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_k, bar(C::B_KF + st), ch * 64, hk,
-                      j * BN, b);
+          tma_load_4d(base + C::OFF_K + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_k, bar(C::B_KF + st),
+                      ch * C::CH_ELEMS, hk, j * BN, b);
         ++k_issued;
       }
       // Drain: every issued copy must land before shared memory is released.
@@ -228,8 +245,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_VF + st), C::KV_BYTES);
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_4d(base + C::OFF_V + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_v, bar(C::B_VF + st), ch * 64, hk,
-                      j * BN, b);
+          tma_load_4d(base + C::OFF_V + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_v, bar(C::B_VF + st),
+                      ch * C::CH_ELEMS, hk, j * BN, b);
         ++v_issued;
       }
       for (int j = max(0, v_issued - VST); j < v_issued; ++j) mbar_wait_drain(bar(C::B_VF + j % VST), (j / VST) & 1);
@@ -240,8 +257,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // The whole warp runs the schedule (descriptors stay warp-uniform); one
     // elected lane issues each tcgen05 instruction, predicated (no branch).
     const bool leader = elect_one();
-    constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+    constexpr uint32_t idesc_s = C::FP8 ? idesc_e4m3_f32(128, BN, false) : idesc_bf16_f32(128, BN, false);
+    constexpr uint32_t idesc_o = C::FP8 ? idesc_e4m3_f32(128, D, true) : idesc_bf16_f32(128, D, true);
     bool ok = true;
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -263,11 +280,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
       const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        // advance the start-address field (16-byte units) to k-step ks
+      for (int ks = 0; ks < D / C::K_MMA; ++ks) {
+        // advance the start-address field (16-byte units) to k-step ks (32 bytes of a row)
         const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
         const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
-        mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+        if constexpr (C::FP8) mma_ss_f8(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+        else mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
       }
       mma_commit(bar(C::B_SF + t * NSL + (j % NSL)), leader);
       if (t == last_tile(j)) mma_commit(bar(C::B_KE + st), leader);
@@ -296,9 +314,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
         const uint64_t vdesc = sdesc_sw128(base + C::OFF_V + st * C::KV_BYTES, C::KV_CHUNK, 1024);
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          mma_ts(o_tmem, p_tmem + ks * 8, vdesc + ((ks * 16 * 128) >> 4), idesc_o, (j > 0 || ks > 0) ? 1u : 0u,
-                 leader);
+        for (int ks = 0; ks < BN / C::K_MMA; ++ks) {
+          // K_MMA keys per step: 8 TMEM columns of packed P, K_MMA rows of V
+          const uint64_t vd = vdesc + ((ks * C::K_MMA * 128) >> 4);
+          if constexpr (C::FP8) mma_ts_f8(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
+          else mma_ts(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
+        }
         mma_commit(bar(C::B_OD + t), leader);
         if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t), leader);
         if (t == last_tile(j)) mma_commit(bar(C::B_VE + st), leader);
@@ -346,18 +367,24 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
       }
       const float mx = row_max<BN>(s);
       const float m_new = fmaxf(m_run, mx * sl2);
-      const bool grow = m_new > m_run + kRescaleThreshold;
+      const bool grow = m_new > m_run + C::RESCALE_THR;
       const float m_use = grow ? m_new : m_run;
       const float alpha = grow ? ex2(m_run - m_use) : 1.f;
-      const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-      uint32_t p[BN / 2];
+      // p is measured from 2^P_SHIFT below the reference max (l and O carry
+      // the same factor, so O/l is unchanged; the LSE subtracts it again)
+      const float m_eff = ((m_use == -INFINITY) ? 0.f : m_use) - C::P_SHIFT;
+      uint32_t p[C::P_WORDS];
       // Blocks with masked keys use the MUFU exp2 only (masked scores are -inf
       // and must give exactly 0); full blocks send part of the work to the FMA pipe.
-      const float sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
+      float sum;
+      if constexpr (C::FP8)
+        sum = need_mask ? exp_row_e4m3<BN, false>(s, p, sl2, m_eff) : exp_row_e4m3<BN, true>(s, p, sl2, m_eff);
+      else
+        sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
       l_run = l_run * alpha + sum;
       m_run = m_use;
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) tmem_st32(t_tmem + slot * BN + c * 32, p + c * 32);
+      for (int c = 0; c < C::P_WORDS / 32; ++c) tmem_st32(t_tmem + slot * BN + c * 32, p + c * 32);
       tmem_st_wait();
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         // O must hold P_{j-1} V_{j-1} before it is rescaled.  The wait is
@@ -388,9 +415,10 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
       tc_fence_after();
     }
     const bool write = ok && !*abort_flag;
-    const uint32_t stage = base + C::OFF_Q + t * C::Q_BYTES;   // Q tile is dead: reuse it
+    // bf16 O staging: the dead Q tile, or (FP8, whose Q tile is smaller) a region of its own
+    const uint32_t stage = C::FP8 ? base + C::OFF_OST + t * (128 * D * 2) : base + C::OFF_Q + t * C::Q_BYTES;
     if (write) {
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float inv_l = (l_run > 0.f) ? a.o_mul / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -416,12 +444,13 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
     named_bar_sync(1 + t, 128);
     if (write && wq == 0 && lane == 0 && r0 < a.Nq) {
 #pragma unroll
-      for (int ch = 0; ch < C::DCH; ++ch) tma_store_4d(&tm_o, stage + ch * C::Q_CHUNK, ch * 64, hq, r0, b);
+      for (int ch = 0; ch < D / 64; ++ch) tma_store_4d(&tm_o, stage + ch * C::Q_CHUNK, ch * 64, hq, r0, b);   // bf16 O
       tma_store_commit();
       tma_store_wait_read();
     }
     if (write && row < a.Nq)
-      a.lse[((size_t)b * a.Hq + hq) * a.Nq + row] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      a.lse[((size_t)b * a.Hq + hq) * a.Nq + row] =
+          (l_run > 0.f) ? (m_run - C::P_SHIFT + log2f(l_run)) * kLn2 : -INFINITY;
     __syncwarp();
   }
 
@@ -433,10 +462,10 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
-               int Nk, float scale, cudaStream_t stream) {
-  using C = FwdCfg<D, CAUSAL, (D <= 128) ? 128 : 64>;
+               int Nk, float scale, cudaStream_t stream, float qk_descale = 1.f, float v_descale = 1.f) {
+  using C = FwdCfg<D, CAUSAL, (D <= 128) ? 128 : 64, FP8>;
   static int attr_done = 0;
   const void* kfn = reinterpret_cast<const void*>(&attn_fwd_kernel<C>);
   if (int rc = ensure_smem_attr(kfn, C::SMEM_BYTES, &attr_done)) return rc;
@@ -444,14 +473,21 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (!status) return ATTN_ERR_CUDA;
 
   CUtensorMap tq, tk, tv, to;
-  const uint64_t es = 2;
-  const uint32_t box_q[4] = {64, 1, (uint32_t)C::BM, 1};
-  const uint32_t box_kv[4] = {64, 1, (uint32_t)C::BN, 1};
+  const uint64_t es = C::ES;
+  const uint32_t box_q[4] = {(uint32_t)C::CH_ELEMS, 1, (uint32_t)C::BM, 1};
+  const uint32_t box_kv[4] = {(uint32_t)C::CH_ELEMS, 1, (uint32_t)C::BN, 1};
+  auto encode_in = [&](CUtensorMap* m, const void* ptr, const uint64_t* dims, const uint64_t* strides,
+                       const uint32_t* box) {
+    return FP8 ? encode_u8_4d(m, ptr, dims, strides, box) : encode_bf16_4d(m, ptr, dims, strides, box);
+  };
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Nq, (uint64_t)B};
     const uint64_t strides[3] = {D * es, (uint64_t)Hq * D * es, (uint64_t)Nq * Hq * D * es};
-    if (!encode_bf16_4d(&tq, q, dims, strides, box_q)) return ATTN_ERR_CUDA;
-    if (!encode_bf16_4d(&to, o, dims, strides, box_q)) return ATTN_ERR_CUDA;
+    if (!encode_in(&tq, q, dims, strides, box_q)) return ATTN_ERR_CUDA;
+    // O is bf16 in both forms
+    const uint64_t ostrides[3] = {D * 2ull, (uint64_t)Hq * D * 2, (uint64_t)Nq * Hq * D * 2};
+    const uint32_t box_o[4] = {64, 1, (uint32_t)C::BM, 1};
+    if (!encode_bf16_4d(&to, o, dims, ostrides, box_o)) return ATTN_ERR_CUDA;
   }
   {
     // With Nk == 0 no key block is ever loaded: describe a 1-row tensor at q.
@@ -460,8 +496,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const void* vb = Nk > 0 ? v : q;
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, nk, (uint64_t)B};
     const uint64_t strides[3] = {D * es, (uint64_t)Hkv * D * es, nk * Hkv * D * es};
-    if (!encode_bf16_4d(&tk, kb, dims, strides, box_kv)) return ATTN_ERR_CUDA;
-    if (!encode_bf16_4d(&tv, vb, dims, strides, box_kv)) return ATTN_ERR_CUDA;
+    if (!encode_in(&tk, kb, dims, strides, box_kv)) return ATTN_ERR_CUDA;
+    if (!encode_in(&tv, vb, dims, strides, box_kv)) return ATTN_ERR_CUDA;
   }
   FwdArgs a;
   a.lse = lse;
@@ -472,7 +508,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.group = Hq / Hkv;
   a.n_qblk = (Nq + C::BM * C::NT - 1) / (C::BM * C::NT);
   a.causal_off = Nk - Nq;
-  a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale_log2 = scale * qk_descale * 1.4426950408889634f;
+  a.o_mul = v_descale;
   dim3 grid(a.n_qblk, Hq, B);
   attn_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -505,4 +542,26 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     default: return c ? launch_fwd<256, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s)
                       : launch_fwd<256, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s);
   }
+}
+
+extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                            float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int D,
+                            int causal, float scale, void* stream) {
+  using namespace ea;
+  if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 0 || B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  for (float d : {q_descale, k_descale, v_descale})
+    if (!(d > 0.f) || !isfinite(d)) return ATTN_ERR_INVALID_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Nq == 0) return ATTN_OK;
+  if ((uint64_t)B * Nq * Hq * D * 2 >= (1ull << 40) || (uint64_t)B * Nk * Hkv * D >= (1ull << 40))
+    return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float qk = q_descale * k_descale;
+  return causal ? launch_fwd<128, true, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s, qk, v_descale)
+                : launch_fwd<128, false, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s, qk, v_descale);
 }

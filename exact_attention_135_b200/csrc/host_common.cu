@@ -80,6 +80,11 @@ bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], 
   return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, strides, box);
 }
 
+bool encode_u8_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                  const uint32_t box[4]) {
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 4, dims, strides, box);
+}
+
 bool encode_f32_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                    const uint32_t box[4]) {
   return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 4, dims, strides, box);

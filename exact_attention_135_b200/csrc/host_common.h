@@ -23,6 +23,10 @@ int* device_status_ptr();
 bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                     const uint32_t box[4]);
 
+// The same for 8-bit elements (box[0] must be <= 128).
+bool encode_u8_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                  const uint32_t box[4]);
+
 // The same for fp32 elements (box[0] * 4 bytes must be <= 128).
 bool encode_f32_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],
                    const uint32_t box[4]);

@@ -57,4 +57,35 @@ __device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float s
   return (a0 + b0) + (a1 + b1);
 }
 
+// The same with p packed four to a word as e4m3 bytes (column 4w + i in
+// byte i of word w), the layout of an 8-bit A operand in tensor memory.
+template <int N, bool MIXED>
+__device__ __forceinline__ float exp_row_e4m3(const uint32_t* s, uint32_t* p, float sl2, float m) {
+  const uint64_t k2 = f2_pack(sl2, sl2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int c = 0; c < N / 2; ++c) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), k2, nm2);
+    float p0, p1;
+    if (MIXED && poly_pair(c)) {
+      exp2_poly_x2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    if (c & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
+    else acc0 = f2_add(acc0, f2_pack(p0, p1));
+    const uint32_t pair = pack_e4m3x2(p0, p1);
+    if (c & 1) p[c / 2] |= pair << 16;
+    else p[c / 2] = pair;
+  }
+  float a0, a1, b0, b1;
+  f2_unpack(acc0, a0, a1);
+  f2_unpack(acc1, b0, b1);
+  return (a0 + b0) + (a1 + b1);
+}
+
 }  // namespace ea

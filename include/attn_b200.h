@@ -84,6 +84,26 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              int Nk, int D, int Dv, int causal, float scale, void* stream);
 
 /*
+ * attn_fwd_fp8: attn_fwd with e4m3 inputs ("FlashAttention (KO)", section
+ * "FlashAttention-3 (2024)": FP8 support on Hopper).
+ *
+ *   q [B, Nq, Hq, D], k [B, Nk, Hkv, D], v [B, Nk, Hkv, D]: OCP FP8 E4M3 bytes
+ *   q_descale, k_descale, v_descale: per-tensor factors; the represented
+ *       values are q_descale * e4m3(q) and likewise for k and v
+ *   o [B, Nq, Hq, D] bf16 (written), lse [B, Hq, Nq] fp32 (written)
+ *
+ * Computes O = softmax(scale * Q K^T + causal mask) V and the LSE of the
+ * represented values, exactly as attn_fwd defines them.  Q K^T is taken on
+ * the e4m3 tensor cores with fp32 accumulation; each probability is rounded
+ * to e4m3 before the product with V (relative error up to 2^-4), the row sums
+ * and the LSE use the unrounded probabilities.  Supported: D == 128; descales
+ * finite and > 0; the other rules as attn_fwd.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale, float v_descale,
+                 void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int D, int causal, float scale,
+                 void* stream);
+
+/*
  * attn_bwd_workspace_size: bytes of device workspace that attn_bwd needs for
  * B x Nq query rows of Hq heads of width D (an fp32 dQ accumulator plus one
  * fp32 value per query row).  0 for an unsupported D.  The caller allocates

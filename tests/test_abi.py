@@ -132,3 +132,16 @@ def test_bwd_argument_checks(lib):
     need = lib.attn_bwd_workspace_size(1, 4, 100, 128)
     assert need >= 100 * 4 * 128 * 4 + 100 * 4 * 4
     assert lib.attn_bwd_workspace_size(1, 4, 100, 256) == 0
+
+
+def test_fwd_fp8_argument_checks(lib):
+    def call(q=A, D=128, descale=0.01, scale=0.1, Hq=4, Hkv=2):
+        return lib.attn_fwd_fp8(q, A, A, descale, 0.02, 0.03, A, A, 1, Hq, Hkv, 100, 100, D, 1, scale, None)
+    assert call(q=None) == 1
+    assert call(q=A + 8) == 1                # misaligned
+    assert call(descale=0.0) == 1
+    assert call(descale=float("nan")) == 1
+    assert call(scale=-1.0) == 1
+    assert call(Hq=6, Hkv=4) == 1
+    assert call(D=64) == 2
+    assert call(D=256) == 2
