@@ -21,6 +21,12 @@
 // tile while the other tile's softmax runs.  Head dim 256 keeps one tile with
 // two S buffers instead (TMEM holds 128 lanes x 512 fp32 columns: O alone
 // takes 256 of them).
+//
+// FP8 option (attn_fwd_fp8, head dim 128; "FlashAttention (KO)", section
+// "FlashAttention-3 (2024)"): Q, K, V tiles hold E4M3 bytes, both products
+// run as kind::f8f6f4 MMAs (32 bytes = 32 elements of reduction per MMA), P is
+// rounded to e4m3 and packed four to a TMEM column, and the Q/K descales are
+// folded into the score scale and the V descale into the epilogue.
 #include <math.h>
 
 #include "host_common.h"

@@ -1,12 +1,16 @@
 /*
  * attn_b200.h: C ABI of the B200 (sm_100a) fused exact-attention library.
  *
- * Two operations, both computing  O = softmax(scale * Q K^T + mask) V  and the
- * per-row log-sum-exp, exactly (up to floating-point rounding), without ever
- * writing the score matrix to device memory:
+ * Operations computing  O = softmax(scale * Q K^T + mask) V  and the per-row
+ * log-sum-exp, exactly (up to floating-point rounding), without ever writing
+ * the score matrix to device memory, and the gradients of the forward:
  *
- *   attn_fwd           prefill / training forward over dense Q, K, V
- *   attn_decode_paged  one-token MLA ("MQA-absorb") decode over a paged cache
+ *   attn_fwd               prefill / training forward over dense Q, K, V
+ *   attn_fwd_fp8           the same on E4M3 inputs with per-tensor descales
+ *   attn_bwd               dQ, dK, dV of attn_fwd, recomputing S and P
+ *   attn_decode_paged      one-token MLA ("MQA-absorb") decode over a paged cache
+ *   attn_decode_paged_mtp  the same with s_q query tokens per sequence
+ *   attn_decode_paged_gqa  one-token decode over paged, grouped K and V caches
  *
  * Sources for what is computed (web pages, cited by title and section):
  *   - "FlashAttention (KO)", section on the problems of standard attention:
