@@ -53,7 +53,8 @@ tests/test_oracle_mtp.py pin the GQA-path and multi-token decode functions
 with brute forces, closed forms, invariances and planted mistakes;
 tests/test_oracle_fp8.py pins the E4M3 decoding against torch's float8_e4m3fn,
 hand-derived codes and planted mistakes;
-tests/test_oracle_bwd.py pins the gradients with central finite differences
+tests/test_oracle_bwd.py pins the gradients with hand-derived cases
+(tests/golden/hand_worked_bwd.json), central finite differences
 of the forward function, torch fp64 autograd, closed forms, the zero sum of
 the dK rows and planted mistakes.
 """

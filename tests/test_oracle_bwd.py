@@ -1,7 +1,7 @@
 """Pins for the backward oracle (oracle.attention_bwd), CPU only.
 
 The gradients are checked against things other than the function itself:
-central finite differences of the forward oracle (the derivative by its
+hand-derived cases (tests/golden/hand_worked_bwd.json), central finite differences of the forward oracle (the derivative by its
 definition, no backward formula involved), torch autograd through fp64
 scaled_dot_product_attention (independent library code), closed forms for a
 single key and for the last key of a causal square problem, and the
@@ -12,6 +12,9 @@ checks that the pins catch each one.
 
 import importlib
 import inspect
+import json
+import math
+import os
 import textwrap
 
 import numpy as np
@@ -22,6 +25,40 @@ import oracle
 
 # the package re-exports the function `attention`, which shadows the submodule name
 oracle_attention = importlib.import_module("oracle.attention")
+
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_bwd.json")
+
+
+def _val(x):
+    if isinstance(x, (int, float)):
+        return float(x)
+    sgn = -1.0 if x.startswith("-") else 1.0
+    x = x.lstrip("-")
+    if x == "ln3":
+        return sgn * math.log(3.0)
+    if x == "3ln3/4":
+        return sgn * 3.0 * math.log(3.0) / 4.0
+    raise ValueError(x)
+
+
+def _arr(nested):
+    return np.vectorize(_val, otypes=[np.float64])(np.array(nested, dtype=object))
+
+
+with open(GOLDEN) as f:
+    _G = json.load(f)["bwd"]
+
+
+def _golden_check(fn, case):
+    g = fn(_arr(case["q"]), _arr(case["k"]), _arr(case["v"]), _arr(case["do"]), case["causal"], case["scale"])
+    for got, key in zip(g, ("dq", "dk", "dv")):
+        np.testing.assert_allclose(got, _arr(case[key]), rtol=0, atol=1e-14, err_msg=f"{case['name']} {key}")
+
+
+@pytest.mark.parametrize("case", _G, ids=[c["name"] for c in _G])
+def test_hand_worked_cases(case):
+    _golden_check(oracle.attention_bwd, case)
 
 
 def _rand(shape, rng):
@@ -201,6 +238,7 @@ def test_pins_catch_planted_mistakes(name):
     checks = [lambda c=c: _fd_check(fn, c) for c in FD_CASES]
     checks += [lambda c=c: _torch_check(fn, c) for c in (False, True)]
     checks += [lambda: _single_key_check(fn), lambda: _last_key_check(fn)]
+    checks += [lambda c=c: _golden_check(fn, c) for c in _G]
     checks += [lambda c=c: _dk_sum_check(fn, c) for c in (False, True)]
     failures = 0
     for chk in checks:
