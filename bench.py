@@ -6,6 +6,11 @@ One step is one pass of the hot path over one batch of synthetic inputs
 already resident in device memory:
   * prefill: attn_fwd on the long-context GQA causal workload
     (B=1, Hq=32, Hkv=8, N=16384, D=128, bf16, scale 1/sqrt(128));
+  * prefill_c4: attn_fwd on the MQA wide-head workload (B=4, Hq=16, Hkv=1,
+    N=4096, D=256, non-causal, Q doubled for peaked rows);
+  * prefill_c2 / prefill_c1: attn_fwd on the GPT-2-small-shaped causal
+    workload (B=8, H=12, N=1024, D=64) and on the tiny one (B=1, H=2, N=128,
+    D=64), both latency-bound at these sizes;
   * decode:  attn_decode_paged on the MLA absorbed paged-decode workload
     (64 sequences x 128 heads, latent 576/512, 64-token pages, lengths
     uniform on [1024, 8192]);
@@ -20,7 +25,9 @@ The headline metric is prefill TFLOP/s (4*Nq*Nk*D per head, halved for
 causal); the decode KV-cache GB/s (bytes of the K/V rows of valid tokens
 over the time of the decode + combine kernels) is reported in the "decode"
 and "gqa_decode" objects of the same line.  All are compared with the
-measured B200 peaks.
+measured B200 peaks.  Every part reports the mean, median and best of its
+per-launch times, and the line ends with a compact "summary" object that
+holds each part's headline figure and roofline fraction.
 
 With N > 1 (torchrun, one process per GPU) every rank runs the same
 independent workload (weak scaling, no collective on the data path); the
@@ -165,8 +172,8 @@ class Part:
         return sum(a.numel() * a.element_size() for a, _ in pairs)
 
 
-def prefill_part(ea, dev):
-    cfg = inputs.PREFILL_CONFIGS[PREFILL_ID]
+def prefill_part(ea, dev, cfg_id=PREFILL_ID, name="prefill"):
+    cfg = inputs.PREFILL_CONFIGS[cfg_id]
     q, k, v = inputs.prefill_config_inputs(cfg)
     host = {"q": q.pin_memory(), "k": k.pin_memory(), "v": v.pin_memory()}
     d = {n: t.to(dev) for n, t in host.items()}
@@ -178,7 +185,7 @@ def prefill_part(ea, dev):
     def run():
         ea.fwd(d["q"], d["k"], d["v"], causal=cfg.causal, scale=cfg.scale, out=d["o"], lse=d["lse"])
 
-    p = Part("prefill", run, [(d[n], host[n]) for n in ("q", "k", "v")],
+    p = Part(name, run, [(d[n], host[n]) for n in ("q", "k", "v")],
              [(host["o"], d["o"]), (host["lse"], d["lse"])], launches=1)
     p.cfg = cfg
     p.work = cfg.flops()
@@ -372,19 +379,18 @@ def run_gpu(args):
     peaks, peaks_kind = load_peaks()
     stream = torch.cuda.current_stream(dev)
 
-    parts = []
-    if args.part in ("all", "prefill"):
-        parts.append(prefill_part(ea, dev))
-    if args.part in ("all", "decode"):
-        parts.append(decode_part(ea, dev))
-    if args.part in ("all", "gqa"):
-        parts.append(gqa_part(ea, dev))
-    if args.part in ("all", "mtp"):
-        parts.append(mtp_part(ea, dev))
-    if args.part in ("all", "fp8"):
-        parts.append(fp8_part(ea, dev))
-    if args.part in ("all", "bwd"):
-        parts.append(bwd_part(ea, dev))
+    builders = [("prefill", lambda: prefill_part(ea, dev)),
+                ("prefill_c4", lambda: prefill_part(ea, dev, 4, "prefill_c4")),
+                ("prefill_c2", lambda: prefill_part(ea, dev, 2, "prefill_c2")),
+                ("decode", lambda: decode_part(ea, dev)),
+                ("prefill_c1", lambda: prefill_part(ea, dev, 1, "prefill_c1")),
+                ("gqa", lambda: gqa_part(ea, dev)),
+                ("mtp", lambda: mtp_part(ea, dev)),
+                ("fp8", lambda: fp8_part(ea, dev)),
+                ("bwd", lambda: bwd_part(ea, dev))]
+    # The small workloads (1 and 2) fit in L2; in the step they run right after
+    # parts that stream 200-400 MB, which evicts them between their launches.
+    parts = [make() for name, make in builders if args.part in ("all", name)]
 
     for _ in range(args.warmup):
         for p in parts:
@@ -407,160 +413,129 @@ def run_gpu(args):
         raise RuntimeError("device status error in timed region")
     e2e = time_e2e(parts, args.e2e_steps, 3, dev, stream)
 
-    # max over ranks of every timing
+    # max over ranks of every timing (mean, median and best per launch, e2e mean)
     names = [p.name for p in parts]
-    vec = [total_ms / args.steps] + [statistics.mean(per[n]) for n in names] + \
-          [statistics.mean(e2e[n]) for n in names]
+    vec = [total_ms / args.steps]
+    for n in names:
+        vec += [statistics.mean(per[n]), statistics.median(per[n]), min(per[n]), statistics.mean(e2e[n])]
     vec = max_over_ranks(vec, device=dev)
     step_ms = vec[0]
-    launch_ms = dict(zip(names, vec[1:1 + len(names)]))
-    e2e_ms = dict(zip(names, vec[1 + len(names):]))
+    stat = {n: dict(zip(("mean", "median", "best", "e2e"), vec[1 + 4 * i:5 + 4 * i])) for i, n in enumerate(names)}
     by = {p.name: p for p in parts}
+
+    sustained = step_ms * args.steps * 1e-3 > SUSTAINED_AFTER_S
+    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    bf16_kind = f"{peaks_kind} bf16 {'sustained' if sustained else 'burst'}"
+
+    def timing(n):
+        t = stat[n]
+        return {"ms_mean": round(t["mean"], 4), "ms_median": round(t["median"], 4), "ms_best": round(t["best"], 4)}
+
+    def e2e_obj(p, work, unit, scale):
+        return {"value": round(world * work / (stat[p.name]["e2e"] * 1e-3) / scale, 2), "unit": unit,
+                "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)}
+
+    def tensor_obj(p, metric, kernel, peak, peak_kind, traffic=None):
+        tf = p.work / (stat[p.name]["mean"] * 1e-3) / 1e12
+        return {"metric": metric, "value": round(whole_job_rate(world, p.work, stat[p.name]["mean"]) / 1e12, 2),
+                "unit": "TFLOP/s", **timing(p.name),
+                "tflops_median": round(p.work / (stat[p.name]["median"] * 1e-3) / 1e12, 2),
+                "config": {"workload": p.cfg.name, "causal": p.cfg.causal},
+                "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                             "frac": round(tf / peak, 4), "peak_kind": peak_kind, "traffic": traffic,
+                             "kernel": kernel, "frac_of_burst": round(tf / peaks["bf16_tflops"], 4)},
+                "e2e": e2e_obj(p, p.work, "TFLOP/s", 1e12)}
+
+    def hbm_obj(p, metric, kernel, traffic=None, extra=None):
+        sec = stat[p.name]["mean"] * 1e-3
+        gbs = p.kv_bytes / sec / 1e9
+        o = {"metric": metric, "value": round(whole_job_rate(world, p.kv_bytes, stat[p.name]["mean"]) / 1e9, 1),
+             "unit": "GB/s", **timing(p.name), "gbs_median": round(p.kv_bytes / (stat[p.name]["median"] * 1e-3) / 1e9, 1),
+             "config": {"workload": p.cfg.name, "kv_bytes": p.kv_bytes, "tokens": p.tokens},
+             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
+                          "traffic": traffic, "kernel": kernel},
+             "e2e": e2e_obj(p, p.kv_bytes, "GB/s", 1e9)}
+        if hasattr(p, "flops"):
+            o["roofline"]["tflops"] = round(p.flops / sec / 1e12, 1)
+        if extra:
+            o.update(extra)
+        return o
+
+    objs = {}
+    if "prefill_c4" in by:
+        objs["prefill_c4"] = tensor_obj(by["prefill_c4"], "attention TFLOP/s (prefill, MQA D=256)",
+                                        "attn_fwd_kernel<D=256,non-causal>", bf16_peak, bf16_kind,
+                                        NCU_TRAFFIC_BYTES.get("prefill_c4"))
+    if "prefill_c2" in by:
+        objs["prefill_c2"] = tensor_obj(by["prefill_c2"], "attention TFLOP/s (prefill, GPT-2-small shape)",
+                                        "attn_fwd_kernel<D=64,causal>", bf16_peak, bf16_kind)
+    if "prefill_c1" in by:
+        p = by["prefill_c1"]
+        o = tensor_obj(p, "attention TFLOP/s (prefill, tiny)", "attn_fwd_kernel<D=64,non-causal>", bf16_peak,
+                       bf16_kind)
+        o["us_per_call"] = round(stat[p.name]["mean"] * 1e3, 2)
+        objs["prefill_c1"] = o
+    if "decode" in by:
+        objs["decode"] = hbm_obj(by["decode"], "KV-cache GB/s (paged MLA decode)",
+                                 "decode_split_kernel + decode_combine_kernel", NCU_TRAFFIC_BYTES.get("decode"),
+                                 {"workspace_bytes": by["decode"].ws_bytes})
+    if "gqa" in by:
+        objs["gqa_decode"] = hbm_obj(by["gqa"], "KV-cache GB/s (GQA-path paged decode)",
+                                     "gqa_decode_kernel + gqa_combine_kernel", NCU_TRAFFIC_BYTES.get("gqa"))
+    if "mtp" in by:
+        p = by["mtp"]
+        extra = {"s_q": MTP_SQ, "query_tokens_per_s": round(world * p.cfg.B * MTP_SQ / (stat["mtp"]["mean"] * 1e-3), 1)}
+        if "decode" in by:
+            extra["time_vs_one_token"] = round(stat["mtp"]["mean"] / stat["decode"]["mean"], 3)
+        objs["decode_mtp"] = hbm_obj(p, f"KV-cache GB/s (paged MLA decode, {MTP_SQ} query tokens per sequence)",
+                                     "decode kernels over query units", NCU_TRAFFIC_BYTES.get("mtp"), extra)
+    if "fp8" in by:
+        # no measured fp8 peak: the measured bf16 peak times the nominal dense fp8/bf16 ratio (4.5 / 2.25)
+        o = tensor_obj(by["fp8"], "attention TFLOP/s (FP8 E4M3 prefill)", "attn_fwd_kernel<D=128,causal,fp8>",
+                       2.0 * bf16_peak, bf16_kind + " x 2 (nominal fp8/bf16 ratio)", NCU_TRAFFIC_BYTES.get("fp8"))
+        o["roofline"]["frac_of_bf16_peak"] = o["roofline"].pop("frac_of_burst")
+        objs["fp8"] = o
+    if "bwd" in by:
+        o = tensor_obj(by["bwd"], "attention backward TFLOP/s",
+                       "bwd_prep_kernel + attn_bwd_kernel<D=128,causal> + bwd_dq_kernel (timed together)",
+                       bf16_peak, bf16_kind, NCU_TRAFFIC_BYTES.get("bwd"))
+        o["config"]["flops"] = "2.5 x forward (five products)"
+        objs["bwd"] = o
 
     line = {"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: i.i.d. N(0,1) bf16 from a seeded CPU generator",
             "gpu_launches": args.steps * sum(p.launches for p in parts), "clocks": clocks}
     step_parts = "+".join(names)
-    decode_obj = None
-    if "decode" in by:
-        p = by["decode"]
-        gbs = p.kv_bytes / (launch_ms["decode"] * 1e-3) / 1e9
-        decode_obj = {
-            "metric": "KV-cache GB/s (paged decode)",
-            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["decode"]) / 1e9, 1), "unit": "GB/s",
-            "ms_per_launch": round(launch_ms["decode"], 4),
-            "config": {"workload": p.cfg.name, "B": p.cfg.B, "Hq": p.cfg.Hq, "Dk": p.cfg.Dk, "Dv": p.cfg.Dv,
-                       "page_size": p.cfg.page_size, "lengths": f"uniform [{p.cfg.min_len}, {p.cfg.max_len}]",
-                       "tokens": p.tokens, "kv_bytes": p.kv_bytes, "scale": p.cfg.scale,
-                       "l2": "KV cache 340 MB per step, larger than L2, no flush"},
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
-                         "traffic": NCU_TRAFFIC_BYTES["decode"], "kernel": "decode_split_kernel + decode_combine_kernel",
-                         "tflops": round(p.flops / (launch_ms["decode"] * 1e-3) / 1e12, 1),
-                         "tensor_frac": round(p.flops / (launch_ms["decode"] * 1e-3) / 1e12 /
-                                              peaks["bf16_tflops"], 4)},
-            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["decode"] * 1e-3) / 1e9, 1), "unit": "GB/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-            "workspace_bytes": p.ws_bytes,
-        }
-    gqa_obj = None
-    if "gqa" in by:
-        p = by["gqa"]
-        gbs = p.kv_bytes / (launch_ms["gqa"] * 1e-3) / 1e9
-        gqa_obj = {
-            "metric": "KV-cache GB/s (GQA-path paged decode)",
-            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["gqa"]) / 1e9, 1), "unit": "GB/s",
-            "ms_per_launch": round(launch_ms["gqa"], 4),
-            "config": {"workload": p.cfg.name, "B": p.cfg.B, "Hq": p.cfg.Hq, "Hkv": p.cfg.Hkv, "D": p.cfg.D,
-                       "page_size": p.cfg.page_size, "lengths": f"uniform [{p.cfg.min_len}, {p.cfg.max_len}]",
-                       "tokens": p.tokens, "kv_bytes": p.kv_bytes, "scale": p.cfg.scale,
-                       "l2": "K/V cache 1.35 GB per step, larger than L2, no flush"},
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
-                         "traffic": NCU_TRAFFIC_BYTES["gqa"], "kernel": "gqa_decode_kernel + gqa_combine_kernel"},
-            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["gqa"] * 1e-3) / 1e9, 1), "unit": "GB/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-            "workspace_bytes": p.ws_bytes,
-        }
-    mtp_obj = None
-    if "mtp" in by:
-        p = by["mtp"]
-        sec = launch_ms["mtp"] * 1e-3
-        mtp_obj = {
-            "metric": f"KV-cache GB/s (paged MLA decode, {MTP_SQ} query tokens per sequence)",
-            "value": round(whole_job_rate(world, p.kv_bytes, launch_ms["mtp"]) / 1e9, 1), "unit": "GB/s",
-            "ms_per_launch": round(launch_ms["mtp"], 4),
-            "query_tokens_per_s": round(world * p.cfg.B * MTP_SQ / sec, 1),
-            "config": {"workload": p.cfg.name + f", s_q={MTP_SQ}", "s_q": MTP_SQ, "kv_bytes": p.kv_bytes,
-                       "attended_positions": p.pairs},
-            "roofline": {"bound": "hbm", "achieved": round(p.kv_bytes / sec / 1e9, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(p.kv_bytes / sec / 1e9 / peaks["hbm_gbs"], 4),
-                         "peak_kind": f"{peaks_kind} HBM copy", "traffic": None,
-                         "kernel": "decode_split_kernel + decode_combine_kernel (query units)",
-                         "tflops": round(p.flops / sec / 1e12, 1)},
-            "e2e": {"value": round(world * p.kv_bytes / (e2e_ms["mtp"] * 1e-3) / 1e9, 1), "unit": "GB/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-        }
-    sustained = step_ms * args.steps * 1e-3 > SUSTAINED_AFTER_S
-    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    bf16_kind = f"{peaks_kind} bf16 {'sustained' if sustained else 'burst'}"
-    fp8_obj = None
-    if "fp8" in by:
-        p = by["fp8"]
-        tf = p.work / (launch_ms["fp8"] * 1e-3) / 1e12
-        # no measured fp8 peak: the measured bf16 peak times the nominal dense fp8/bf16 ratio (4.5 / 2.25)
-        fp8_peak = 2.0 * bf16_peak
-        fp8_obj = {
-            "metric": "attention TFLOP/s (FP8 E4M3 prefill)",
-            "value": round(whole_job_rate(world, p.work, launch_ms["fp8"]) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_launch": round(launch_ms["fp8"], 4),
-            "config": {"workload": p.cfg.name + ", E4M3 inputs with per-tensor descales", "dtype": "e4m3"},
-            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(tf / fp8_peak, 4), "peak_kind": bf16_kind + " x 2 (nominal fp8/bf16 ratio)",
-                         "traffic": NCU_TRAFFIC_BYTES["fp8"], "kernel": "attn_fwd_kernel<D=128,causal,fp8>",
-                         "frac_of_bf16_peak": round(tf / bf16_peak, 4)},
-            "e2e": {"value": round(world * p.work / (e2e_ms["fp8"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-        }
-    bwd_obj = None
-    if "bwd" in by:
-        p = by["bwd"]
-        tf = p.work / (launch_ms["bwd"] * 1e-3) / 1e12
-        bwd_obj = {
-            "metric": "attention backward TFLOP/s",
-            "value": round(whole_job_rate(world, p.work, launch_ms["bwd"]) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_launch": round(launch_ms["bwd"], 4),
-            "config": {"workload": "backward of " + p.cfg.name, "flops": "2.5 x forward (five products)",
-                       "workspace_bytes": p.ws_bytes},
-            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16_peak, "unit": "TFLOP/s",
-                         "frac": round(tf / bf16_peak, 4), "peak_kind": bf16_kind, "traffic": NCU_TRAFFIC_BYTES["bwd"],
-                         "kernel": "bwd_prep_kernel + attn_bwd_kernel<D=128,causal> + bwd_dq_kernel (timed together)",
-                         "frac_of_burst": round(tf / peaks["bf16_tflops"], 4)},
-            "e2e": {"value": round(world * p.work / (e2e_ms["bwd"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-        }
     if "prefill" in by:
         p = by["prefill"]
-        achieved = p.work / (launch_ms["prefill"] * 1e-3) / 1e12
-        sustained = step_ms * args.steps * 1e-3 > SUSTAINED_AFTER_S
-        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-        line.update({
-            "metric": "attention TFLOP/s (prefill)",
-            "value": round(whole_job_rate(world, p.work, launch_ms["prefill"]) / 1e12, 2),
-            "unit": "TFLOP/s",
-            "config": {"workload": p.cfg.name, "step": step_parts, "B": p.cfg.B, "Hq": p.cfg.Hq,
-                       "Hkv": p.cfg.Hkv, "Nq": p.cfg.Nq, "Nk": p.cfg.Nk, "D": p.cfg.D, "causal": p.cfg.causal,
-                       "scale": p.cfg.scale, "global_batch": p.cfg.B * world, "seq_len": p.cfg.Nq,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (Q 134 MB + K/V 67 MB per step), no flush"},
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4),
-                         "peak_kind": f"{peaks_kind} bf16 {'sustained' if sustained else 'burst'}",
-                         "traffic": NCU_TRAFFIC_BYTES["prefill"], "kernel": "attn_fwd_kernel<D=128,causal>",
-                         "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-                         "algorithmic_bytes": p.cfg.io_bytes()},
-            "e2e": {"value": round(world * p.work / (e2e_ms["prefill"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": p.bytes(p.h2d), "d2h_bytes_per_step": p.bytes(p.d2h)},
-        })
-        if decode_obj:
-            line["decode"] = decode_obj
-        if gqa_obj:
-            line["gqa_decode"] = gqa_obj
-        if mtp_obj:
-            line["decode_mtp"] = mtp_obj
-        if fp8_obj:
-            line["fp8"] = fp8_obj
-        if bwd_obj:
-            line["bwd"] = bwd_obj
+        head = tensor_obj(p, "attention TFLOP/s (prefill)", "attn_fwd_kernel<D=128,causal>", bf16_peak, bf16_kind,
+                          NCU_TRAFFIC_BYTES["prefill"])
+        head["roofline"]["algorithmic_bytes"] = p.cfg.io_bytes()
+        head["config"] = {"workload": p.cfg.name, "step": step_parts, "B": p.cfg.B, "Hq": p.cfg.Hq,
+                          "Hkv": p.cfg.Hkv, "Nq": p.cfg.Nq, "Nk": p.cfg.Nk, "D": p.cfg.D, "causal": p.cfg.causal,
+                          "global_batch": p.cfg.B * world, "seq_len": p.cfg.Nq, "parallelism": f"replicas x{world}",
+                          "l2": "inputs larger than L2 (Q 134 MB + K/V 67 MB per step), no flush"}
     else:
-        head = decode_obj or gqa_obj or mtp_obj or fp8_obj or bwd_obj
-        line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
-        line["config"]["step"] = step_parts
-        if decode_obj and gqa_obj:
-            line["gqa_decode"] = gqa_obj
+        head = next(iter(objs.values()))
+        head["config"]["step"] = step_parts
+    line.update({k: head[k] for k in ("metric", "value", "unit", "config", "roofline", "e2e")})
+    line.update({k: head[k] for k in ("ms_mean", "ms_median", "ms_best")})
+    line.update(objs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and "prefill" in by:
         line["cpu_baseline"] = cpu_baseline(args.baseline_rows)
+    # last key: one figure and one roofline fraction per part, short enough to
+    # survive any truncation of the line's head
+    summary = {}
+    if "prefill" in by:
+        summary["prefill_c3"] = [head["value"], head["roofline"]["frac"]]
+    for k, o in objs.items():
+        summary[k] = [o["value"], o["roofline"]["frac"]]
+    if "decode_mtp" in objs and "time_vs_one_token" in objs["decode_mtp"]:
+        summary["mtp_time_vs_one_token"] = objs["decode_mtp"]["time_vs_one_token"]
+    summary["units"] = "prefill/fp8/bwd TFLOP/s, decodes GB/s; [value, roofline frac]"
+    line["summary"] = summary
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -657,7 +632,8 @@ def main():
     ap.add_argument("--baseline-rows", type=int, default=768,
                     help="query rows per head in the cpu_baseline sample (about 10 s of CPU work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", choices=["all", "prefill", "decode", "gqa", "mtp", "fp8", "bwd"], default="all",
+    ap.add_argument("--part", choices=["all", "prefill", "prefill_c4", "prefill_c2", "prefill_c1", "decode", "gqa",
+                                       "mtp", "fp8", "bwd"], default="all",
                     help="time only one piece of the step (for profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end (host buffer) timing")
     args = ap.parse_args()

@@ -48,14 +48,14 @@ _SIGNATURES = {
     "attn_abi_version": (_i, []),
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
-    "attn_decode_paged_workspace_size": (_sz, [_i, _i, _i]),
+    "attn_decode_paged_workspace_size": (_sz, [_i, _i, _i, _i]),
     "attn_decode_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_read_device_status": (_i, [_i]),
     "attn_decode_paged_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_decode_paged_noalloc_max_bytes": (_sz, []),
     "attn_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
-    "attn_decode_paged_gqa_workspace_size": (_sz, [_i, _i, _i, _i]),
-    "attn_decode_paged_mtp_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_decode_paged_gqa_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_decode_paged_mtp_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode_paged_mtp": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _f, _f, _f, _vp, _vp] + [_i] * 7 + [_f, _vp]),
@@ -220,9 +220,18 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     return dq, dk, dv
 
 
+def _device_index(device) -> int:
+    if device is None:
+        return torch.cuda.current_device()
+    if isinstance(device, int):
+        return device
+    d = torch.device(device)
+    return d.index if d.index is not None else torch.cuda.current_device()
+
+
 def decode_workspace_size(B: int, Hq: int, Dv: int, device=None) -> int:
-    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        return int(library().attn_decode_paged_workspace_size(B, Hq, Dv))
+    """Workspace bytes of decode_paged on `device` (0: unsupported shape or device)."""
+    return int(library().attn_decode_paged_workspace_size(B, Hq, Dv, _device_index(device)))
 
 
 def decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
@@ -249,7 +258,7 @@ def decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Ten
     _need(out, "out", torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 2)
     with torch.cuda.device(q.device):
-        need = int(library().attn_decode_paged_workspace_size(B, Hq, dv))
+        need = int(library().attn_decode_paged_workspace_size(B, Hq, dv, q.device.index))
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
         if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
@@ -264,8 +273,8 @@ def decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Ten
 
 
 def decode_mtp_workspace_size(B: int, s_q: int, Hq: int, Dv: int, device=None) -> int:
-    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        return int(library().attn_decode_paged_mtp_workspace_size(B, s_q, Hq, Dv))
+    """Workspace bytes of decode_paged_mtp on `device` (0: unsupported shape or device)."""
+    return int(library().attn_decode_paged_mtp_workspace_size(B, s_q, Hq, Dv, _device_index(device)))
 
 
 def decode_paged_mtp(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
@@ -293,7 +302,7 @@ def decode_paged_mtp(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch
     _need(out, "out", torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 3)
     with torch.cuda.device(q.device):
-        need = int(library().attn_decode_paged_mtp_workspace_size(B, sq, Hq, dv))
+        need = int(library().attn_decode_paged_mtp_workspace_size(B, sq, Hq, dv, q.device.index))
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
         if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
@@ -337,8 +346,8 @@ def decode_paged_noalloc(q: torch.Tensor, kv_pages: torch.Tensor, block_table: t
 
 
 def decode_gqa_workspace_size(B: int, Hq: int, Hkv: int, D: int, device=None) -> int:
-    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        return int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D))
+    """Workspace bytes of decode_paged_gqa on `device` (0: unsupported shape or device)."""
+    return int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D, _device_index(device)))
 
 
 def decode_paged_gqa(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
@@ -367,7 +376,7 @@ def decode_paged_gqa(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tens
     _need(out, "out", torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 2)
     with torch.cuda.device(q.device):
-        need = int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D))
+        need = int(library().attn_decode_paged_gqa_workspace_size(B, Hq, Hkv, D, q.device.index))
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
         if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:

@@ -593,24 +593,21 @@ inline WsLayout ws_layout(int B, int pairs) {
   return w;
 }
 
-inline int pairs_for_device() {
-  const int sms = current_sm_count();
-  return sms >= 2 ? sms / 2 : 0;
-}
+inline int pairs_for_sms(int sms) { return sms >= 2 ? sms / 2 : 0; }
 
 }  // namespace dec
 }  // namespace ea
 
-extern "C" size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv) {
+extern "C" size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv, int device) {
   using namespace ea::dec;
   if (B < 1 || s_q < 1 || (long long)B * s_q > B_MAX || Hq != HQ || Dv != DV) return 0;
-  const int pairs = pairs_for_device();
-  if (pairs == 0) return 0;
+  const int pairs = pairs_for_sms(ea::sm_count_of(device));
+  if (pairs == 0 || pairs > MAX_PARTS) return 0;
   return ws_layout(B * s_q, pairs).total;
 }
 
-extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv) {
-  return attn_decode_paged_mtp_workspace_size(B, 1, Hq, Dv);
+extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv, int device) {
+  return attn_decode_paged_mtp_workspace_size(B, 1, Hq, Dv, device);
 }
 
 extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const int32_t* block_table,
@@ -631,7 +628,7 @@ extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const 
   const int units = B * s_q;
   if ((long long)num_pages * PAGE >= (1ll << 31) || (long long)B * max_pages_per_seq >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
-  const int pairs = pairs_for_device();
+  const int pairs = pairs_for_sms(current_sm_count());
   if (pairs == 0) return ATTN_ERR_CUDA;
   if (pairs > MAX_PARTS) return ATTN_ERR_UNSUPPORTED;
   const WsLayout wl = ws_layout(units, pairs);
@@ -742,7 +739,9 @@ extern "C" int attn_decode_paged_noalloc(const void* q, const void* kv_pages, co
                                          int Dv, int page_size, int num_pages, int max_pages_per_seq, float scale,
                                          void* stream) {
   using namespace ea::dec;
-  const size_t need = attn_decode_paged_workspace_size(B, Hq, Dv);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const size_t need = attn_decode_paged_workspace_size(B, Hq, Dv, dev);
   if (need > kNoAllocScratchBytes) return ATTN_ERR_UNSUPPORTED;   // batch too large for the fixed array
   void* scratch = noalloc_scratch();
   if (!scratch) return ATTN_ERR_CUDA;

@@ -502,13 +502,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // One CTA per (sequence, KV head): merges the partial results of a unit that
 // several workers shared, writes O = 0 and LSE = -inf for an empty sequence,
 // leaves units written by the decode kernel untouched.  The number of pieces
-// is not bounded: weights are recomputed from the LSEs on the fly.
+// is not bounded: they are taken in chunks of COMBINE_CHUNK, and each chunk's
+// slots and weights are computed once into shared memory, so the loop over
+// output elements only reads them.
 constexpr int COMBINE_THREADS = 128;
+constexpr int COMBINE_CHUNK = 128;
+constexpr int COMBINE_OUT = 8;   // output elements per thread: G * D <= 8 * 128
 
 __global__ void __launch_bounds__(COMBINE_THREADS) gqa_combine_kernel(const Args a) {
   const int b = blockIdx.x, g = blockIdx.y;
   const int G = a.G, D = a.D, Hq = a.Hkv * G;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = a.Hkv * a.ws_pref[a.B];
   const int np = a.ws_pref[b + 1] - a.ws_pref[b];
   if (np == 0) {
@@ -520,40 +524,95 @@ __global__ void __launch_bounds__(COMBINE_THREADS) gqa_combine_kernel(const Args
   const int u0 = a.Hkv * a.ws_pref[b] + g * np, u1 = u0 + np;
   const int w_lo = worker_of_page(u0, T, a.workers), w_hi = worker_of_page(u1 - 1, T, a.workers);
   if (w_lo == w_hi) return;
+  const int n = w_hi - w_lo + 1;
   // slot of worker w's piece of this unit (workers with empty ranges hold none)
   auto slot_of = [&](int w) -> int {
     const int r0 = range_start(w, T, a.workers);
     if (range_start(w + 1, T, a.workers) == r0) return -1;
     return 2 * w + ((w == w_lo && u0 != r0) ? 1 : 0);
   };
+  __shared__ float s_red[COMBINE_THREADS / 32][8];
   __shared__ float s_max[8], s_inv[8];
-  if (tid < G) {
-    float mx = -INFINITY;
-    for (int w = w_lo; w <= w_hi; ++w) {
-      const int s = slot_of(w);
-      if (s >= 0) mx = fmaxf(mx, a.ws_lse[(size_t)s * G + tid]);
+  __shared__ int s_slot[COMBINE_CHUNK];
+  __shared__ float s_w[8][COMBINE_CHUNK];
+
+  // per-head maximum, then sum of exp(lse - max), over all pieces (in parallel over pieces)
+  for (int pass = 0; pass < 2; ++pass) {
+    float acc[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) acc[h] = pass == 0 ? -INFINITY : 0.f;
+    for (int i = tid; i < n; i += COMBINE_THREADS) {
+      const int sl = slot_of(w_lo + i);
+      if (sl < 0) continue;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h >= G) break;
+        const float l = a.ws_lse[(size_t)sl * G + h];
+        if (pass == 0) acc[h] = fmaxf(acc[h], l);
+        else if (s_max[h] != -INFINITY) acc[h] += expf(l - s_max[h]);
+      }
     }
-    float sum = 0.f;
-    for (int w = w_lo; w <= w_hi; ++w) {
-      const int s = slot_of(w);
-      if (s >= 0 && mx != -INFINITY) sum += expf(a.ws_lse[(size_t)s * G + tid] - mx);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float v = acc[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float y = __shfl_xor_sync(0xffffffffu, v, o);
+        v = pass == 0 ? fmaxf(v, y) : v + y;
+      }
+      if (lane == 0) s_red[warp][h] = v;
     }
-    s_max[tid] = mx;
-    s_inv[tid] = sum > 0.f ? 1.f / sum : 0.f;
-    a.lse[(size_t)b * Hq + g * G + tid] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    __syncthreads();
+    if (tid < G) {
+      float v = s_red[0][tid];
+      for (int w = 1; w < COMBINE_THREADS / 32; ++w) v = pass == 0 ? fmaxf(v, s_red[w][tid]) : v + s_red[w][tid];
+      if (pass == 0) {
+        s_max[tid] = v;
+      } else {
+        s_inv[tid] = v > 0.f ? 1.f / v : 0.f;
+        a.lse[(size_t)b * Hq + g * G + tid] = v > 0.f ? s_max[tid] + logf(v) : -INFINITY;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int i = tid; i < G * D; i += COMBINE_THREADS) {
-    const int h = i / D, d = i % D;
-    const float mx = s_max[h], inv = s_inv[h];
-    float acc = 0.f;
-    for (int w = w_lo; w <= w_hi; ++w) {
-      const int s = slot_of(w);
-      if (s < 0 || mx == -INFINITY) continue;
-      const float wgt = expf(a.ws_lse[(size_t)s * G + h] - mx) * inv;
-      acc += wgt * a.ws_o[((size_t)s * G + h) * D + d];
+
+  // O = sum over pieces of weight * partial O, one chunk of pieces at a time
+  float out[COMBINE_OUT];
+#pragma unroll
+  for (int k = 0; k < COMBINE_OUT; ++k) out[k] = 0.f;
+  for (int c0 = 0; c0 < n; c0 += COMBINE_CHUNK) {
+    const int cn = min(COMBINE_CHUNK, n - c0);
+    if (tid < cn) {
+      const int sl = slot_of(w_lo + c0 + tid);
+      s_slot[tid] = sl;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h >= G) break;
+        s_w[h][tid] = (sl < 0 || s_max[h] == -INFINITY)
+                          ? 0.f
+                          : expf(a.ws_lse[(size_t)sl * G + h] - s_max[h]) * s_inv[h];
+      }
     }
-    a.o[((size_t)b * Hq + g * G + h) * D + d] = __float2bfloat16(acc);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < COMBINE_OUT; ++k) {
+      const int i = tid + k * COMBINE_THREADS;
+      if (i >= G * D) break;
+      const int h = i / D;
+      float acc = out[k];
+      for (int j = 0; j < cn; ++j) {
+        const int sl = s_slot[j];
+        if (sl >= 0) acc += s_w[h][j] * a.ws_o[(size_t)sl * G * D + i];
+      }
+      out[k] = acc;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int k = 0; k < COMBINE_OUT; ++k) {
+    const int i = tid + k * COMBINE_THREADS;
+    if (i >= G * D) break;
+    a.o[((size_t)b * Hq + g * G) * D + i] = __float2bfloat16(out[k]);
   }
 }
 
@@ -587,13 +646,13 @@ int launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, int ctas
 }  // namespace gqa
 }  // namespace ea
 
-extern "C" size_t attn_decode_paged_gqa_workspace_size(int B, int Hq, int Hkv, int D) {
+extern "C" size_t attn_decode_paged_gqa_workspace_size(int B, int Hq, int Hkv, int D, int device) {
   using namespace ea;
   using namespace ea::gqa;
   if (B < 1 || B > B_MAX || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
-  const int sms = current_sm_count();
+  const int sms = sm_count_of(device);
   if (sms < 1) return 0;
   return ws_layout(B, G, D, sms * workers_per_cta(D)).total;
 }

@@ -63,9 +63,8 @@ int* device_status_ptr() {
   return g_status_ptr[dev];
 }
 
-int current_sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+int sm_count_of(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 0;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_sm_count[dev]) {
     int n = 0;
@@ -73,6 +72,12 @@ int current_sm_count() {
     g_sm_count[dev] = n;
   }
   return g_sm_count[dev];
+}
+
+int current_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return sm_count_of(dev);
 }
 
 bool encode_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const uint64_t strides[3],

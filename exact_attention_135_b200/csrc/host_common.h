@@ -44,6 +44,9 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 // Raise the dynamic shared-memory limit of a kernel once per device.
 int ensure_smem_attr(const void* kernel, int bytes, int* done_mask);
 
+// Streaming multiprocessors of the current device, or of device `dev`
+// (0 if the device does not exist or CUDA fails).
 int current_sm_count();
+int sm_count_of(int dev);
 
 }  // namespace ea

@@ -139,10 +139,11 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Nq, int D);
  * attn_fwd.  Supported: D == Dv in {64, 128}; Hq % Hkv == 0; scale finite and
  * > 0; tensors 16-byte aligned, lse 4-byte aligned.  Accumulation is fp32; P
  * and dS are rounded to bf16 before their products; outputs are rounded to
- * bf16 once.  dk and dv are deterministic run to run; dq is accumulated with
- * fp32 atomic adds (one per key block), so its last bits may vary from run
- * to run.  Returns ATTN_ERR_WORKSPACE if the workspace is missing, too small
- * or misaligned.
+ * bf16 once.  dk and dv are deterministic run to run; dq is summed over key
+ * blocks in an fp32 accumulator (each key block's contribution is added at L2
+ * by a TMA reduce-add of a shared-memory tile, in whatever order the CTAs
+ * reach it), so its last bits may vary from run to run.  Returns
+ * ATTN_ERR_WORKSPACE if the workspace is missing, too small or misaligned.
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int D, int Dv, int causal,
@@ -151,9 +152,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
 /*
  * attn_decode_paged_workspace_size: bytes of device workspace that
  * attn_decode_paged needs for a batch of B sequences with Hq heads of width
- * Dv on the current device.  The caller allocates it (any alignment >= 256 B).
+ * Dv when it runs on CUDA device `device` (the split-KV plan depends on the
+ * device's SM count).  Returns 0 for an unsupported shape, or when `device`
+ * is not a valid CUDA device index.  The caller allocates it, 256-byte
+ * aligned, on that device.
  */
-size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv);
+size_t attn_decode_paged_workspace_size(int B, int Hq, int Dv, int device);
 
 /*
  * attn_decode_paged: one new query token per sequence attending to a paged
@@ -190,9 +194,10 @@ int attn_decode_paged(const void* q, const void* kv_pages, const int32_t* block_
 
 /*
  * attn_decode_paged_mtp_workspace_size: workspace bytes of attn_decode_paged_mtp
- * for B sequences with s_q query tokens each (0 for an unsupported shape).
+ * for B sequences with s_q query tokens each on CUDA device `device` (0 for an
+ * unsupported shape or an invalid device index).
  */
-size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv);
+size_t attn_decode_paged_mtp_workspace_size(int B, int s_q, int Hq, int Dv, int device);
 
 /*
  * attn_decode_paged_mtp: attn_decode_paged with s_q >= 1 new query tokens per
@@ -229,7 +234,9 @@ int attn_decode_paged_mtp(const void* q, const void* kv_pages, const int32_t* bl
  * attn_decode_paged_noalloc_max_bytes() bytes (40 MiB), held on every GPU
  * that loads the library until the process exits; a batch whose workspace
  * (attn_decode_paged_workspace_size) exceeds it is rejected with
- * ATTN_ERR_UNSUPPORTED before anything is enqueued.  The call allocates no
+ * ATTN_ERR_UNSUPPORTED before anything is enqueued.  The workspace grows with
+ * the device's SM count; on a 148-SM B200 every batch up to the decode's
+ * limit of 2048 sequences fits, so there only that limit applies.  The call allocates no
  * device memory.  The first call on each device looks up the array's device
  * address (with that device current), so make it before any stream capture.
  * All calls share the array and it keeps the last call's contents: calls whose
@@ -246,9 +253,10 @@ size_t attn_decode_paged_noalloc_max_bytes(void);
 /*
  * attn_decode_paged_gqa_workspace_size: bytes of device workspace that
  * attn_decode_paged_gqa needs for B sequences, Hq query heads in groups of
- * Hq / Hkv, head dim D, on the current device (0 for an unsupported shape).
+ * Hq / Hkv, head dim D, on CUDA device `device` (0 for an unsupported shape or
+ * an invalid device index).
  */
-size_t attn_decode_paged_gqa_workspace_size(int B, int Hq, int Hkv, int D);
+size_t attn_decode_paged_gqa_workspace_size(int B, int Hq, int Hkv, int D, int device);
 
 /*
  * attn_decode_paged_gqa: one new query token per sequence attending to a

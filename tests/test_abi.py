@@ -108,7 +108,7 @@ def test_mtp_decode_argument_checks(lib):
     assert call(scale=-1.0) == 1
     assert call(Hq=64) == 2
     assert call(B=1024, s_q=4) == 2          # more than 2048 query units
-    assert lib.attn_decode_paged_mtp_workspace_size(1024, 4, 128, 512) == 0
+    assert lib.attn_decode_paged_mtp_workspace_size(1024, 4, 128, 512, 0) == 0
 
 
 def test_bwd_argument_checks(lib):
@@ -145,3 +145,15 @@ def test_fwd_fp8_argument_checks(lib):
     assert call(Hq=6, Hkv=4) == 1
     assert call(D=64) == 2
     assert call(D=256) == 2
+
+
+def test_workspace_sizes_reject_bad_device_index(lib):
+    # the split plan depends on the SM count of the device the call will run on;
+    # a device index that names no CUDA device gives 0 (no GPU is needed for this)
+    for dev in (-1, 4096):
+        assert lib.attn_decode_paged_workspace_size(64, 128, 512, dev) == 0
+        assert lib.attn_decode_paged_mtp_workspace_size(64, 2, 128, 512, dev) == 0
+        assert lib.attn_decode_paged_gqa_workspace_size(64, 32, 8, 128, dev) == 0
+    # unsupported shapes give 0 whatever the device
+    assert lib.attn_decode_paged_workspace_size(64, 64, 512, 0) == 0
+    assert lib.attn_decode_paged_gqa_workspace_size(64, 32, 8, 96, 0) == 0

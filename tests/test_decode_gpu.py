@@ -145,6 +145,11 @@ def test_workspace_checks():
     q, kv, bt, sl = _dev(c)
     need = ea.decode_workspace_size(2, HQ, DV)
     assert need > 0
+    lib = ea.library()
+    # the size is that of the device named by the call's device argument
+    assert lib.attn_decode_paged_workspace_size(2, HQ, DV, 0) == need
+    assert lib.attn_decode_paged_workspace_size(2, HQ, DV, torch.cuda.device_count()) == 0
+    assert lib.attn_decode_paged_workspace_size(2, HQ, DV, -1) == 0
     small = torch.empty(need - 256, dtype=torch.uint8, device=q.device)
     with pytest.raises(ValueError):
         ea.decode_paged(q, kv, bt, sl, SCALE, workspace=small)
