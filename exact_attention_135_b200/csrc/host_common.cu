@@ -67,8 +67,19 @@ int sm_count_of(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return 0;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_sm_count[dev]) {
+    // A query about a device that does not exist must not leave an error
+    // behind for the next launch's cudaGetLastError check: validate the index
+    // first and clear whatever a failed query records.
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess || dev >= count) {
+      (void)cudaGetLastError();
+      return 0;
+    }
     int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return 0;
+    }
     g_sm_count[dev] = n;
   }
   return g_sm_count[dev];
