@@ -22,12 +22,26 @@
 // SM, so the two CTAs of a pair split the 512 output columns: CTA r owns
 // columns [256 r, 256 r + 256).  Each CTA computes the full 128 x 64 score
 // tile per page itself.  TMEM columns per CTA:
-//   [0,256) O half | [256,320) S | [320,352) P (bf16) | [352,512) Q dims 256..575
-// Q dims 0..255 sit in shared memory (64 KB) next to a 2-stage ring of whole
-// pages (2 x 72 KB).
+//   [0,256) O half | [256,320) S buffer 0 | [320,384) S buffer 1 | [384,512) Q dims 320..575
+// Score tiles alternate between the two S buffers, so the tile of page g+1
+// is computed while the softmax still reads that of page g; P (bf16) is
+// written over the first 32 columns of its own S buffer.  Q dims 0..319 sit
+// in shared memory (80 KB).
+//
+// A page's latent rows reach shared memory in two parts with rings of their
+// own, each filled by its own producer warp:
+//   own part   the 4 column chunks (256 dims) of this CTA's output columns:
+//              read by the score MMAs and then by the P V products;
+//   rest part  the other CTA's 256 dims and the 64 RoPE dims (5 chunks): read
+//              by the score MMAs only.
+// The score MMAs take the rest chunks first and release them with a commit,
+// then the own chunks; so a rest slot is free ~800 cycles before the score
+// tile is complete, and an own part has to land only when the score MMAs reach
+// it.  A whole-page stage would be held from its load until the P V product.
 #include <math.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "host_common.h"
 #include "sm100.cuh"
@@ -42,36 +56,58 @@ constexpr int DK = 576;
 constexpr int DV = 512;
 constexpr int PAGE = 64;
 constexpr int B_MAX = 2048;
-constexpr int STAGES = 2;
 constexpr int CHUNKS = DK / 64;                 // 9 column chunks of 128 bytes
-constexpr int Q_SMEM_CHUNKS = 4;                // dims 0..255 in shared memory
-constexpr int Q_TMEM_DIMS = DK - 64 * Q_SMEM_CHUNKS;   // 320 dims in TMEM
+constexpr int Q_SMEM_CHUNKS = 5;                // dims 0..319 in shared memory
+constexpr int Q_TMEM_DIMS = DK - 64 * Q_SMEM_CHUNKS;   // 256 dims in TMEM
 constexpr int Q_CHUNK_BYTES = HQ * 128;         // 16 KB
 constexpr int PAGE_CHUNK_BYTES = PAGE * 128;    // 8 KB
 constexpr int Q_BYTES = Q_SMEM_CHUNKS * Q_CHUNK_BYTES;
-constexpr int STAGE_BYTES = CHUNKS * PAGE_CHUNK_BYTES;  // 72 KB
-static_assert(STAGE_BYTES == PAGE * DK * 2, "a stage holds exactly one page of the pool");
+constexpr int OWN_CHUNKS = 4;                   // this CTA's 256 output dims
+constexpr int REST_CHUNKS = CHUNKS - OWN_CHUNKS;   // the other CTA's 256 dims + 64 RoPE dims
+constexpr int OWN_BYTES = OWN_CHUNKS * PAGE_CHUNK_BYTES;     // 32 KB
+constexpr int REST_BYTES = REST_CHUNKS * PAGE_CHUNK_BYTES;   // 40 KB
+static_assert(OWN_BYTES + REST_BYTES == PAGE * DK * 2, "the two parts hold exactly one page of the pool");
+// The rest part has one slot, released chunk by chunk: chunk j of page g+1 is
+// asked for as soon as the score MMAs of page g have read chunk j of page g
+// (a commit per chunk), so each 8 KB chunk has about one page period to land.
+// Own parts are held until the P V product and get three stages.
+constexpr int OWN_STAGES = 3;
+constexpr int REST_STAGES = 1;
 constexpr int O_COL = 0;
-constexpr int S_COL = 256;
-constexpr int P_COL = 320;
-constexpr int Q_COL = 352;
+constexpr int S_COL = 256;                      // two buffers of PAGE columns
+constexpr int Q_COL = 384;
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 224;                    // 4 softmax warps, producer, two MMA issuers
-constexpr int PRODUCER_WARP = 4;
+constexpr int THREADS = 256;                    // 4 softmax warps, 2 producers, 2 MMA issuers
+constexpr int REST_PRODUCER_WARP = 4;           // Q and the rest parts (and the L2 prefetches)
 constexpr int MMA_S_WARP = 5;                   // score tiles S = Q K^T
 constexpr int MMA_PV_WARP = 6;                  // products O += P V
+constexpr int OWN_PRODUCER_WARP = 7;            // the own parts
 // barriers
-constexpr int B_QF = 0, B_QE = 1, B_QT = 2, B_KF = 3, B_KE = B_KF + STAGES, B_SF = B_KE + STAGES;
-constexpr int B_SE = B_SF + 1, B_PF = B_SE + 1, B_OD = B_PF + 1, B_DR = B_OD + 1, B_DRS = B_DR + 1;
+constexpr int B_QF = 0, B_QE = 1, B_QT = 2;
+constexpr int B_RF = 3;                          // rest part landed (one arrival per chunk)
+constexpr int B_RE = B_RF + 1;                   // rest chunk j read, one barrier per chunk
+constexpr int B_OF = B_RE + REST_CHUNKS, B_OE = B_OF + OWN_STAGES;
+constexpr int B_SF = B_OE + OWN_STAGES;         // score tile complete, one per S buffer
+constexpr int B_SB = B_SF + 2;                   // P V product done, one per S buffer (its P is read)
+constexpr int B_PF = B_SB + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, B_DRS = B_DR + 1;
 constexpr int NBAR = B_DRS + 1;
 // shared memory
 constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + Q_BYTES;
-constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
+constexpr int OFF_OWN = OFF_Q + Q_BYTES;
+constexpr int OFF_REST = OFF_OWN + OWN_STAGES * OWN_BYTES;
+constexpr int OFF_BAR = OFF_REST + REST_STAGES * REST_BYTES;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int OFF_PREF = OFF_MISC + 16;
 constexpr int SMEM_BYTES = OFF_PREF + (B_MAX + 1) * 4 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(OFF_OWN % 1024 == 0 && OFF_REST % 1024 == 0 && REST_BYTES % 1024 == 0, "swizzle atoms");
+static_assert(REST_STAGES == 1, "the rest slot is released chunk by chunk");
+
+// Dim chunk (64 dims) held by chunk j of the own / rest part of CTA `half`.
+__device__ __forceinline__ int own_chunk_dim(int half, int j) { return OWN_CHUNKS * half + j; }
+__device__ __forceinline__ int rest_chunk_dim(int half, int j) {
+  return j < OWN_CHUNKS ? OWN_CHUNKS * (1 - half) + j : CHUNKS - 1;
+}
 
 // Pages the producer asks L2 for ahead of the page it loads: a page's TMA
 // load is issued only when a stage frees up, and from HBM it takes ~2000
@@ -185,12 +221,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bar(B_QF), 1);
     mbar_init(bar(B_QE), 1);
     mbar_init(bar(B_QT), 4);
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar(B_KF + s), 1);
-      mbar_init(bar(B_KE + s), 1);
+    mbar_init(bar(B_RF), REST_CHUNKS);
+    for (int j = 0; j < REST_CHUNKS; ++j) mbar_init(bar(B_RE + j), 1);
+    for (int s = 0; s < OWN_STAGES; ++s) {
+      mbar_init(bar(B_OF + s), 1);
+      mbar_init(bar(B_OE + s), 1);
     }
-    mbar_init(bar(B_SF), 1);
-    mbar_init(bar(B_SE), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_SF + i), 1);
+      mbar_init(bar(B_SB + i), 1);
+    }
     mbar_init(bar(B_PF), 4);
     mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_DR), 1);
@@ -222,7 +262,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) pref[0] = 0;
     if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
   }
-  if (warp == PRODUCER_WARP && lane == 0) {
+  if (warp == REST_PRODUCER_WARP && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kv);
   }
@@ -239,8 +279,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = threadIdx.x; i <= a.B; i += THREADS) a.ws_pref[i] = pref[i];
   const int R0 = range_start(pair, T, a.pairs), R1 = range_start(pair + 1, T, a.pairs);
 
-  if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
+  if (warp == REST_PRODUCER_WARP) {
+    // ------------------------------------------------------------ Q and rest-part producer
     if (lane == 0) {
       SegWalk w;
       w.init(pref, a.B, R0, R1);
@@ -258,7 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto prefetch_next = [&]() {
         if (!p_more) return;
         const int page = a.block_table[(size_t)(p_b / a.s_q) * a.max_pages + (p_gp - pref[p_b])];
-        if (page >= 0 && page < a.num_pages) l2_prefetch(a.kv + (size_t)page * STAGE_BYTES, STAGE_BYTES);
+        if (page >= 0 && page < a.num_pages) l2_prefetch(a.kv + (size_t)page * (PAGE * DK * 2), PAGE * DK * 2);
         if (++p_gp == p_g1) {
           p_more = wp.next(p_b, p_g0, p_g1);
           if (p_more) p_gp = p_g0;
@@ -278,29 +318,62 @@ __global__ void __launch_bounds__(THREADS, 1)
             atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
             page = 0;   // never read outside the pool; the result of this sequence is undefined
           }
-          const int st = g % STAGES;
-          if (!mbar_wait(bar(B_KE + st), ((g / STAGES) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(B_KF + st), STAGE_BYTES);
-          for (int ch = 0; ch < CHUNKS; ++ch)
-            tma_load_2d(base + OFF_KV + st * STAGE_BYTES + ch * PAGE_CHUNK_BYTES, &tm_kv, bar(B_KF + st), ch * 64,
-                         page * PAGE);
+          for (int j = 0; j < REST_CHUNKS && ok; ++j) {
+            if (!mbar_wait(bar(B_RE + j), (g & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(B_RF), PAGE_CHUNK_BYTES);
+            tma_load_2d(base + OFF_REST + j * PAGE_CHUNK_BYTES, &tm_kv, bar(B_RF), rest_chunk_dim(half, j) * 64,
+                        page * PAGE);
+          }
+          if (!ok) break;
           ++issued;
           prefetch_next();
         }
         ++seg;
       }
-      for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait_drain(bar(B_KF + j % STAGES), (j / STAGES) & 1);
+      // the last page's chunks (a page whose loads were cut short by an abort
+      // never completes its phase; the drain wait is bounded)
+      if (issued > 0) mbar_wait_drain(bar(B_RF), (issued - 1) & 1);
       if (q_last >= 0) mbar_wait_drain(bar(B_QF), q_last & 1);
+    }
+    __syncwarp();
+  } else if (warp == OWN_PRODUCER_WARP) {
+    // ------------------------------------------------------------ own-part producer
+    // Waits only for the P V product that frees its slot, never behind a
+    // rest part, so each own part is asked for as soon as its slot is free.
+    if (lane == 0) {
+      SegWalk w;
+      w.init(pref, a.B, R0, R1);
+      int sb, g0, g1, g = 0;
+      bool ok = true;
+      int issued = 0;
+      while (ok && w.next(sb, g0, g1)) {
+        const int32_t* row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages;
+        for (int gp = g0; gp < g1; ++gp, ++g) {
+          int page = row[gp - pref[sb]];
+          if (page < 0 || page >= a.num_pages) page = 0;   // recorded by the rest producer
+          const int st = g % OWN_STAGES;
+          if (!mbar_wait(bar(B_OE + st), ((g / OWN_STAGES) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(B_OF + st), OWN_BYTES);
+          for (int j = 0; j < OWN_CHUNKS; ++j)
+            tma_load_2d(base + OFF_OWN + st * OWN_BYTES + j * PAGE_CHUNK_BYTES, &tm_kv, bar(B_OF + st),
+                        own_chunk_dim(half, j) * 64, page * PAGE);
+          ++issued;
+        }
+      }
+      for (int j = max(0, issued - OWN_STAGES); j < issued; ++j)
+        mbar_wait_drain(bar(B_OF + j % OWN_STAGES), (j / OWN_STAGES) & 1);
     }
     __syncwarp();
   } else if (warp == MMA_S_WARP) {
     // ------------------------------------------------------------ score MMA issuer
     // Two warps issue MMAs, each waiting only for what its own products need:
-    // this one S = Q K^T per page (page landed, S buffer read by the softmax),
-    // the next one O += P V (P written).  A P V product therefore never waits
-    // behind the next page's load, and it frees the page's stage as early as
-    // possible.  S, P and O occupy disjoint TMEM columns, so the two issue
-    // streams need no ordering between them beyond those barriers.
+    // this one S = Q K^T per page (page parts landed, S buffer read by the
+    // softmax), the next one O += P V (P written).  A P V product therefore
+    // never waits behind the next page's load.  S, P and O occupy disjoint
+    // TMEM columns, so the two issue streams need no ordering between them
+    // beyond those barriers.
+    // The 36 k-steps of a score tile take the rest part's chunks first; a
+    // commit then frees the rest slot while the own chunks are multiplied.
     // Warp-uniform schedule; one elected lane issues (predicated, no branch).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
@@ -309,26 +382,51 @@ __global__ void __launch_bounds__(THREADS, 1)
     int sb, g0, g1, seg = 0, g = 0;
     bool ok = true;
     const uint64_t qdesc = sdesc_sw128(base + OFF_Q, 16, 1024);
+    // The k-steps of the chunks of one part, fully unrolled for this CTA's
+    // half so that every descriptor is the part's base plus a constant (the
+    // issue rate of these N=64 products is what bounds the score tile).
+    auto part_mmas = [&](auto half_c, auto rest_c, uint32_t d_tmem, uint64_t kdesc) {
+      constexpr int H = decltype(half_c)::value;
+      constexpr bool REST = decltype(rest_c)::value;
+      constexpr int NCH = REST ? REST_CHUNKS : OWN_CHUNKS;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int c = REST ? (j < OWN_CHUNKS ? OWN_CHUNKS * (1 - H) + j : CHUNKS - 1) : OWN_CHUNKS * H + j;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint32_t acc = (REST && j == 0 && k4 == 0) ? 0u : 1u;
+          const uint64_t kd = kdesc + ((j * PAGE_CHUNK_BYTES + k4 * 32) >> 4);
+          if (c < Q_SMEM_CHUNKS)
+            mma_ss(d_tmem, qdesc + ((c * Q_CHUNK_BYTES + k4 * 32) >> 4), kd, idesc_s, acc, leader);
+          else
+            mma_ts(d_tmem, tmem + Q_COL + ((c - Q_SMEM_CHUNKS) * 4 + k4) * 8, kd, idesc_s, acc, leader);
+        }
+        if (REST) mma_commit(bar(B_RE + j), leader);   // rest chunk j may be refilled
+      }
+    };
     while (ok && w.next(sb, g0, g1)) {
       if (!warp_wait(bar(B_QF), seg & 1, abort_flag, a.status)) break;
       if (!warp_wait(bar(B_QT), seg & 1, abort_flag, a.status)) break;
       for (int gp = g0; gp < g1; ++gp, ++g) {
-        const int st = g % STAGES;
-        if (!warp_wait(bar(B_KF + st), (g / STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
-        if (g > 0 && !warp_wait(bar(B_SE), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        const int os = g % OWN_STAGES, sbuf = g & 1;
+        const uint32_t s_tmem = tmem + S_COL + sbuf * PAGE;
+        if (!warp_wait(bar(B_RF), g & 1, abort_flag, a.status)) { ok = false; break; }
+        // S buffer `sbuf` last held page g-2, whose P the P V product of page
+        // g-2 reads; that product (and with it the softmax's read of S) must be
+        // done.  Pages complete in order, and page g itself cannot complete
+        // before this issue, so the per-buffer barrier is never two phases ahead.
+        if (g >= 2 && !warp_wait(bar(B_SB + sbuf), ((g >> 1) - 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t kdesc = sdesc_sw128(base + OFF_KV + st * STAGE_BYTES, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t dk = ((ks >> 2) * PAGE_CHUNK_BYTES + (ks & 3) * 32) >> 4;
-          if (ks < Q_SMEM_CHUNKS * 4) {
-            const uint32_t dq = ((ks >> 2) * Q_CHUNK_BYTES + (ks & 3) * 32) >> 4;
-            mma_ss(tmem + S_COL, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
-          } else {
-            mma_ts(tmem + S_COL, tmem + Q_COL + (ks - Q_SMEM_CHUNKS * 4) * 8, kdesc + dk, idesc_s, 1u, leader);
-          }
-        }
-        mma_commit(bar(B_SF), leader);
+        const uint64_t rdesc = sdesc_sw128(base + OFF_REST, 16, 1024);
+        if (half == 0) part_mmas(std::integral_constant<int, 0>(), std::true_type(), s_tmem, rdesc);
+        else part_mmas(std::integral_constant<int, 1>(), std::true_type(), s_tmem, rdesc);
+        __syncwarp();
+        if (!warp_wait(bar(B_OF + os), (g / OWN_STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t odesc = sdesc_sw128(base + OFF_OWN + os * OWN_BYTES, 16, 1024);
+        if (half == 0) part_mmas(std::integral_constant<int, 0>(), std::false_type(), s_tmem, odesc);
+        else part_mmas(std::integral_constant<int, 1>(), std::false_type(), s_tmem, odesc);
+        mma_commit(bar(B_SF + sbuf), leader);
         if (gp == g1 - 1) mma_commit(bar(B_QE), leader);   // last score tile of the segment: Q may be replaced
         __syncwarp();
       }
@@ -345,7 +443,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // segment's epilogue has read O (same softmax warps, in order), so the
     // overwrite of O by that page's product needs no extra barrier.  S of a
     // page is complete before its P exists, so this warp's completion of
-    // P V also means the page's stage is no longer read by any MMA.
+    // P V also means the page's own part is no longer read by any MMA.
     const bool leader = elect_one();
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
     SegWalk w;
@@ -356,15 +454,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int gp = g0; gp < g1; ++gp, ++g) {
         if (!warp_wait(bar(B_PF), g & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        const int st = g % STAGES;
-        const uint64_t vdesc =
-            sdesc_sw128(base + OFF_KV + st * STAGE_BYTES + half * 4 * PAGE_CHUNK_BYTES, PAGE_CHUNK_BYTES, 1024);
+        const int os = g % OWN_STAGES;
+        const uint64_t vdesc = sdesc_sw128(base + OFF_OWN + os * OWN_BYTES, PAGE_CHUNK_BYTES, 1024);
+        const uint32_t p_tmem = tmem + S_COL + (g & 1) * PAGE;   // P over its page's S buffer
 #pragma unroll
         for (int kk = 0; kk < PAGE / 16; ++kk)
-          mma_ts(tmem + O_COL, tmem + P_COL + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
+          mma_ts(tmem + O_COL, p_tmem + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
                  (gp == g0 && kk == 0) ? 0u : 1u, leader);
         mma_commit(bar(B_OD), leader);
-        mma_commit(bar(B_KE + st), leader);
+        mma_commit(bar(B_SB + (g & 1)), leader);
+        mma_commit(bar(B_OE + os), leader);   // the own part's slot is free
         __syncwarp();
       }
     }
@@ -383,7 +482,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int sb, g0, g1, seg = 0, g = 0;
     bool ok = true;
     while (ok && w.next(sb, g0, g1)) {
-      // Q dims 256..575 of this head into TMEM (the previous segment's score
+      // Q dims 320..575 of this head into TMEM (the previous segment's score
       // MMAs are complete: its epilogue waited for its last P V product).
       {
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)sb * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
@@ -409,13 +508,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int first_page = pref[sb];
       float m_run = -INFINITY, l_run = 0.f;
       for (int gp = g0; gp < g1; ++gp, ++g) {
-        if (!warp_wait(bar(B_SF), g & 1, abort_flag, a.status)) { ok = false; break; }
+        const uint32_t s_row = t_row + S_COL + (g & 1) * PAGE;   // this page's S buffer
+        if (!warp_wait(bar(B_SF + (g & 1)), (g >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[PAGE];
-        tmem_ld64_sync(t_row + S_COL, s);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_SE));   // S may be overwritten by the next page's scores
+        tmem_ld64_sync(s_row, s);
         const int valid = L - (gp - first_page) * PAGE;   // tokens of this page inside the sequence
         const bool partial = valid < PAGE;
         if (partial) {
@@ -437,7 +534,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         l_run = l_run * alpha + sum;
         m_run = m_use;
         if (gp > g0) {
-          // the previous page's P V product must be complete before P and O change
+          // the previous page's P V product must be complete before O changes
+          // (and before this page's P is announced: the P barrier then never
+          // runs two phases ahead of the P V issuer)
           if (!warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
           if (__any_sync(0xffffffffu, grow)) {
             tc_fence_after();
@@ -451,7 +550,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
-        tmem_st32(t_row + P_COL, p);
+        tmem_st32(s_row, p);   // P over the first PAGE/2 columns of the S just read
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
