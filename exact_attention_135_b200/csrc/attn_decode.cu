@@ -24,9 +24,10 @@
 // tile per page itself.  TMEM columns per CTA:
 //   [0,256) O half | [256,320) S buffer 0 | [320,384) S buffer 1 | [384,512) Q dims 320..575
 // Score tiles alternate between the two S buffers, so the tile of page g+1
-// is computed while the softmax still reads that of page g; P (bf16) is
-// written over the first 32 columns of its own S buffer.  Q dims 0..319 sit
-// in shared memory (80 KB).
+// is computed while the softmax still reads that of page g.  P (bf16) goes to
+// a shared-memory tile (the A operand of the P V product), so an S buffer is
+// free again as soon as the softmax has read it.  Q dims 0..319 sit in shared
+// memory (80 KB).
 //
 // A page's latent rows reach shared memory in two parts with rings of their
 // own, each filled by its own producer warp:
@@ -70,34 +71,53 @@ static_assert(OWN_BYTES + REST_BYTES == PAGE * DK * 2, "the two parts hold exact
 // The rest part has one slot, released chunk by chunk: chunk j of page g+1 is
 // asked for as soon as the score MMAs of page g have read chunk j of page g
 // (a commit per chunk), so each 8 KB chunk has about one page period to land.
-// Own parts are held until the P V product and get three stages.
-constexpr int OWN_STAGES = 3;
+// Own parts are held until the P V product and get two stages: the own part
+// of page g+2 is asked for when the P V product of page g is done, about one
+// page period before the score MMAs of page g+2 reach it.
+constexpr int OWN_STAGES = 2;
 constexpr int REST_STAGES = 1;
 constexpr int O_COL = 0;
 constexpr int S_COL = 256;                      // two buffers of PAGE columns
 constexpr int Q_COL = 384;
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 256;                    // 4 softmax warps, 2 producers, 2 MMA issuers
+// Warps: two softmax groups of four (0-3 and 8-11), two producers, the score
+// MMA issuer and one idle warp.  Each head's row is shared by the two groups
+// (warps w and w+8 reach the same TMEM lanes): group G takes score columns
+// [32G, 32G+32) and output columns [128G, 128G+128) of the CTA's half, so the
+// per-page softmax latency, the rescales and the epilogue are split in two.
+// The groups agree on each row's max through shared memory, and warp 0
+// issues the P V product once both have written their half of P.
+constexpr int THREADS = 384;
 constexpr int REST_PRODUCER_WARP = 4;           // Q and the rest parts (and the L2 prefetches)
 constexpr int MMA_S_WARP = 5;                   // score tiles S = Q K^T
-constexpr int MMA_PV_WARP = 6;                  // products O += P V
 constexpr int OWN_PRODUCER_WARP = 7;            // the own parts
+constexpr int SOFTMAX_THREADS = 256;
+constexpr int BAR_MAX = 1, BAR_P = 2, BAR_L = 3;   // named barriers of the two softmax groups
 // barriers
 constexpr int B_QF = 0, B_QE = 1, B_QT = 2;
 constexpr int B_RF = 3;                          // rest part landed (one arrival per chunk)
 constexpr int B_RE = B_RF + 1;                   // rest chunk j read, one barrier per chunk
 constexpr int B_OF = B_RE + REST_CHUNKS, B_OE = B_OF + OWN_STAGES;
 constexpr int B_SF = B_OE + OWN_STAGES;         // score tile complete, one per S buffer
-constexpr int B_SB = B_SF + 2;                   // P V product done, one per S buffer (its P is read)
-constexpr int B_PF = B_SB + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, B_DRS = B_DR + 1;
+constexpr int B_SB = B_SF + 2;                   // score tile read by the softmax, one per S buffer
+constexpr int B_OD = B_SB + 2, B_DR = B_OD + 1, B_DRS = B_DR + 1;
 constexpr int NBAR = B_DRS + 1;
 // shared memory
 constexpr int OFF_Q = 0;
 constexpr int OFF_OWN = OFF_Q + Q_BYTES;
 constexpr int OFF_REST = OFF_OWN + OWN_STAGES * OWN_BYTES;
-constexpr int OFF_BAR = OFF_REST + REST_STAGES * REST_BYTES;
+// Per softmax warp, a 32 x 128-byte tile through which the segment epilogue
+// transposes O, so that each global store writes whole row pieces.  The
+// first 16 KB also hold P (128 heads x 64 tokens bf16, 128-byte swizzled
+// rows): the epilogue runs only after the segment's last P V product.
+constexpr int XPOSE_BYTES = 32 * 128;
+constexpr int OFF_XPOSE = OFF_REST + REST_STAGES * REST_BYTES;
+constexpr int OFF_P = OFF_XPOSE;
+static_assert(HQ * PAGE * 2 <= 8 * XPOSE_BYTES, "P fits in the transpose tiles");
+constexpr int OFF_BAR = OFF_XPOSE + 8 * XPOSE_BYTES;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_PREF = OFF_MISC + 16;
+constexpr int OFF_XCH = OFF_MISC + 16;          // [2][HQ] floats exchanged by the softmax groups
+constexpr int OFF_PREF = OFF_XCH + 2 * HQ * 4;
 constexpr int SMEM_BYTES = OFF_PREF + (B_MAX + 1) * 4 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(OFF_OWN % 1024 == 0 && OFF_REST % 1024 == 0 && REST_BYTES % 1024 == 0, "swizzle atoms");
@@ -201,6 +221,41 @@ struct SegWalk {
   }
 };
 
+// Block-table entries of the pages of [R0, R1) in order (a page that is
+// not there reads as -1).
+constexpr int LOOKAHEAD = 4;
+static_assert(PREFETCH_PAGES >= 1 && PREFETCH_PAGES < LOOKAHEAD, "prefetch distance within the lookahead");
+struct PageCursor {
+  SegWalk w;
+  const int* pref;
+  const int32_t* row;
+  int gp, g1;
+  bool more;
+  __device__ void init(const int* pref_, const Args& a, int R0, int R1) {
+    pref = pref_;
+    w.init(pref_, a.B, R0, R1);
+    int sb, g0;
+    more = w.next(sb, g0, g1);
+    if (more) {
+      gp = g0;
+      row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages - pref[sb];
+    }
+  }
+  __device__ int next_with(const Args& a) {
+    if (!more) return -1;
+    const int page = row[gp];
+    if (++gp == g1) {
+      int sb, g0;
+      more = w.next(sb, g0, g1);
+      if (more) {
+        gp = g0;
+        row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages - pref[sb];
+      }
+    }
+    return page;
+  }
+};
+
 __global__ void __launch_bounds__(THREADS, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                         const Args a) {
@@ -213,6 +268,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* pref = reinterpret_cast<int*>(base_ptr + OFF_PREF);
   auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8u * i; };
 
+  // Let the combine kernel be scheduled as this grid's CTAs retire (it waits
+  // for this grid's completion before reading anything).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x >> 1;
   const int half = blockIdx.x & 1;
@@ -220,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QF), 1);
     mbar_init(bar(B_QE), 1);
-    mbar_init(bar(B_QT), 4);
+    mbar_init(bar(B_QT), 8);
     mbar_init(bar(B_RF), REST_CHUNKS);
     for (int j = 0; j < REST_CHUNKS; ++j) mbar_init(bar(B_RE + j), 1);
     for (int s = 0; s < OWN_STAGES; ++s) {
@@ -231,26 +289,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(B_SF + i), 1);
       mbar_init(bar(B_SB + i), 1);
     }
-    mbar_init(bar(B_PF), 4);
     mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_DR), 1);
     mbar_init(bar(B_DRS), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // prefix sums of pages per sequence (one pass by warp 0; B <= B_MAX)
+  // Prefix sums of pages per query unit (B <= B_MAX): every thread loads the
+  // lengths of some units at once (one memory latency), then warp 0 scans
+  // them in shared memory.
+  {
+    bool bad = false;
+    for (int u = threadIdx.x; u < a.B; u += THREADS) {
+      const int L = a.seqlens[u / a.s_q];
+      pref[u + 1] = seq_pages(unit_len(a, u), a.max_pages);
+      bad |= (L < 0) || ((long long)L > (long long)a.max_pages * PAGE);
+    }
+    if (bad && blockIdx.x == 0) atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
+  }
+  __syncthreads();
   if (warp == 0) {
     int carry = 0;
-    bool bad = false;
     for (int b0 = 0; b0 < a.B; b0 += 32) {
       const int b = b0 + lane;
-      int n = 0;
-      if (b < a.B) {
-        const int L = a.seqlens[b / a.s_q];
-        n = seq_pages(unit_len(a, b), a.max_pages);
-        bad |= (L < 0) || ((long long)L > (long long)a.max_pages * PAGE);
-      }
-      int x = n;   // inclusive warp scan
+      int x = b < a.B ? pref[b + 1] : 0;   // inclusive warp scan
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -260,7 +322,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       carry += __shfl_sync(0xffffffffu, x, 31);
     }
     if (lane == 0) pref[0] = 0;
-    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
   }
   if (warp == REST_PRODUCER_WARP && lane == 0) {
     tma_prefetch_desc(&tm_q);
@@ -288,32 +349,33 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       int issued = 0;
       int q_last = -1;
-      // A second cursor runs PREFETCH_PAGES pages ahead and prefetches each
-      // page it passes into L2 (one contiguous 72 KB bulk prefetch).
-      SegWalk wp;
-      wp.init(pref, a.B, R0, R1);
-      int p_b = 0, p_g0 = 0, p_g1 = 0, p_gp = 0;
-      bool p_more = wp.next(p_b, p_g0, p_g1);
-      if (p_more) p_gp = p_g0;
-      auto prefetch_next = [&]() {
-        if (!p_more) return;
-        const int page = a.block_table[(size_t)(p_b / a.s_q) * a.max_pages + (p_gp - pref[p_b])];
-        if (page >= 0 && page < a.num_pages) l2_prefetch(a.kv + (size_t)page * (PAGE * DK * 2), PAGE * DK * 2);
-        if (++p_gp == p_g1) {
-          p_more = wp.next(p_b, p_g0, p_g1);
-          if (p_more) p_gp = p_g0;
-        }
-      };
-      for (int i = 0; i < PREFETCH_PAGES; ++i) prefetch_next();
+      // A second cursor runs ahead of the loads and reads the block-table
+      // entries of the next LOOKAHEAD pages into registers (independent loads,
+      // so the first pages cost one memory latency, not one each); each page
+      // is also prefetched into L2 when it is PREFETCH_PAGES ahead of the load.
+      PageCursor cur;
+      cur.init(pref, a, R0, R1);
+      int ids[LOOKAHEAD];
+#pragma unroll
+      for (int i = 0; i < LOOKAHEAD; ++i) ids[i] = cur.next_with(a);
+#pragma unroll
+      for (int i = 0; i < PREFETCH_PAGES; ++i)
+        if (ids[i] >= 0 && ids[i] < a.num_pages) l2_prefetch(a.kv + (size_t)ids[i] * (PAGE * DK * 2), PAGE * DK * 2);
       while (ok && w.next(sb, g0, g1)) {
         if (!mbar_wait(bar(B_QE), (seg & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(bar(B_QF), Q_BYTES);
         for (int ch = 0; ch < Q_SMEM_CHUNKS; ++ch)
           tma_load_2d(base + OFF_Q + ch * Q_CHUNK_BYTES, &tm_q, bar(B_QF), ch * 64, sb * HQ);
         q_last = seg;
-        const int32_t* row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages;
         for (int gp = g0; gp < g1; ++gp, ++g) {
-          int page = row[gp - pref[sb]];
+          int page = ids[0];
+#pragma unroll
+          for (int i = 0; i + 1 < LOOKAHEAD; ++i) ids[i] = ids[i + 1];
+          ids[LOOKAHEAD - 1] = cur.next_with(a);
+          {
+            const int pf = ids[PREFETCH_PAGES - 1];   // the page PREFETCH_PAGES ahead of this one
+            if (pf >= 0 && pf < a.num_pages) l2_prefetch(a.kv + (size_t)pf * (PAGE * DK * 2), PAGE * DK * 2);
+          }
           if (page < 0 || page >= a.num_pages) {
             atomicExch(a.status, (int)ATTN_ERR_INVALID_ARG);
             page = 0;   // never read outside the pool; the result of this sequence is undefined
@@ -326,7 +388,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           if (!ok) break;
           ++issued;
-          prefetch_next();
         }
         ++seg;
       }
@@ -366,14 +427,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == MMA_S_WARP) {
     // ------------------------------------------------------------ score MMA issuer
-    // Two warps issue MMAs, each waiting only for what its own products need:
-    // this one S = Q K^T per page (page parts landed, S buffer read by the
-    // softmax), the next one O += P V (P written).  A P V product therefore
-    // never waits behind the next page's load.  S, P and O occupy disjoint
-    // TMEM columns, so the two issue streams need no ordering between them
-    // beyond those barriers.
-    // The 36 k-steps of a score tile take the rest part's chunks first; a
-    // commit then frees the rest slot while the own chunks are multiplied.
+    // MMAs come from two warps, each waiting only for what its own products
+    // need: this one issues S = Q K^T per page (page parts landed, S buffer
+    // read by the softmax), softmax warp 0 issues O += P V once P is written.
+    // A P V product therefore never waits behind the next page's load.  S and
+    // O occupy disjoint TMEM columns and P lives in shared memory, so the two
+    // issue streams need no ordering between them beyond those barriers.
+    // The 36 k-steps of a score tile take the rest part's chunks first, with a
+    // commit per chunk that lets the producer refill it, then the own chunks.
     // Warp-uniform schedule; one elected lane issues (predicated, no branch).
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, PAGE, false);
@@ -410,10 +471,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int gp = g0; gp < g1; ++gp, ++g) {
         const int os = g % OWN_STAGES, sbuf = g & 1;
         const uint32_t s_tmem = tmem + S_COL + sbuf * PAGE;
+        // the whole rest part (one barrier: waiting chunk by chunk inside the
+        // issue stream slows the score products more than it saves)
         if (!warp_wait(bar(B_RF), g & 1, abort_flag, a.status)) { ok = false; break; }
-        // S buffer `sbuf` last held page g-2, whose P the P V product of page
-        // g-2 reads; that product (and with it the softmax's read of S) must be
-        // done.  Pages complete in order, and page g itself cannot complete
+        // S buffer `sbuf` last held page g-2: the softmax must have read it.
+        // The softmax reads tiles in order, and page g's tile cannot be read
         // before this issue, so the per-buffer barrier is never two phases ahead.
         if (g >= 2 && !warp_wait(bar(B_SB + sbuf), ((g >> 1) - 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
@@ -437,164 +499,216 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
     mbar_wait_drain(bar(B_DRS), 0);
     __syncwarp();
-  } else if (warp == MMA_PV_WARP) {
-    // ------------------------------------------------------------ P V MMA issuer
-    // The P of a segment's first page is written only after the previous
-    // segment's epilogue has read O (same softmax warps, in order), so the
-    // overwrite of O by that page's product needs no extra barrier.  S of a
-    // page is complete before its P exists, so this warp's completion of
-    // P V also means the page's own part is no longer read by any MMA.
-    const bool leader = elect_one();
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
-    SegWalk w;
-    w.init(pref, a.B, R0, R1);
-    int sb, g0, g1, g = 0;
-    bool ok = true;
-    while (ok && w.next(sb, g0, g1)) {
-      for (int gp = g0; gp < g1; ++gp, ++g) {
-        if (!warp_wait(bar(B_PF), g & 1, abort_flag, a.status)) { ok = false; break; }
-        tc_fence_after();
-        const int os = g % OWN_STAGES;
-        const uint64_t vdesc = sdesc_sw128(base + OFF_OWN + os * OWN_BYTES, PAGE_CHUNK_BYTES, 1024);
-        const uint32_t p_tmem = tmem + S_COL + (g & 1) * PAGE;   // P over its page's S buffer
-#pragma unroll
-        for (int kk = 0; kk < PAGE / 16; ++kk)
-          mma_ts(tmem + O_COL, p_tmem + kk * 8, vdesc + ((kk * 16 * 128) >> 4), idesc_o,
-                 (gp == g0 && kk == 0) ? 0u : 1u, leader);
-        mma_commit(bar(B_OD), leader);
-        mma_commit(bar(B_SB + (g & 1)), leader);
-        mma_commit(bar(B_OE + os), leader);   // the own part's slot is free
-        __syncwarp();
-      }
-    }
-    mma_commit(bar(B_DR), leader);
-    __syncwarp();
-    mbar_wait_drain(bar(B_DR), 0);
-    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ idle warp
   } else {
-    // ------------------------------------------------------------ softmax (thread = head)
-    const int h = warp * 32 + lane;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    const uint32_t t_row = tmem + lane_off;
+    // ------------------------------------------------------------ softmax (thread = head, two groups)
+    const int grp = warp >> 3;                  // 0: warps 0-3, 1: warps 8-11
+    const int q4 = warp & 3;
+    const int h = q4 * 32 + lane;
+    const uint32_t t_row = tmem + (uint32_t(q4 * 32) << 16);
+    float* xch = reinterpret_cast<float*>(base_ptr + OFF_XCH);   // [2][HQ]
     const float sl2 = a.scale_log2;
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, true);
+    // Q dims 320..575 of unit u's head into TMEM, half per group; the score
+    // MMAs of segment s+1 wait for it (barrier QT).
+    auto write_q_tmem = [&](int u) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)u * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
+#pragma unroll
+      for (int cc = 0; cc < Q_TMEM_DIMS / 128; ++cc) {
+        const int c = grp * (Q_TMEM_DIMS / 128) + cc;
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(src + c * 8 + i);
+          r[4 * i] = v.x;
+          r[4 * i + 1] = v.y;
+          r[4 * i + 2] = v.z;
+          r[4 * i + 3] = v.w;
+        }
+        tmem_st32(t_row + Q_COL + c * 32, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_QT));
+    };
     SegWalk w;
     w.init(pref, a.B, R0, R1);
     int sb, g0, g1, seg = 0, g = 0;
     bool ok = true;
-    while (ok && w.next(sb, g0, g1)) {
-      // Q dims 320..575 of this head into TMEM (the previous segment's score
-      // MMAs are complete: its epilogue waited for its last P V product).
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)sb * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
-#pragma unroll
-        for (int c = 0; c < Q_TMEM_DIMS / 64; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 u = __ldg(src + c * 8 + i);
-            r[4 * i] = u.x;
-            r[4 * i + 1] = u.y;
-            r[4 * i + 2] = u.z;
-            r[4 * i + 3] = u.w;
-          }
-          tmem_st32(t_row + Q_COL + c * 32, r);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_QT));
-      }
+    bool have = w.next(sb, g0, g1);
+    if (have) write_q_tmem(sb);
+    while (ok && have) {
       const int L = unit_len(a, sb);
       const int first_page = pref[sb];
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f;   // l_run: this group's columns only
       for (int gp = g0; gp < g1; ++gp, ++g) {
         const uint32_t s_row = t_row + S_COL + (g & 1) * PAGE;   // this page's S buffer
-        if (!warp_wait(bar(B_SF + (g & 1)), (g >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        bool good = warp_wait(bar(B_SF + (g & 1)), (g >> 1) & 1, abort_flag, a.status);
         tc_fence_after();
-        uint32_t s[PAGE];
-        tmem_ld64_sync(s_row, s);
-        const int valid = L - (gp - first_page) * PAGE;   // tokens of this page inside the sequence
-        const bool partial = valid < PAGE;
+        uint32_t s[32];
+        tmem_ld32_sync(s_row + grp * 32, s);
+        const int valid = L - (gp - first_page) * PAGE - grp * 32;   // tokens of this half-page in the sequence
+        const bool partial = valid < 32;
         if (partial) {
 #pragma unroll
-          for (int c = 0; c < PAGE; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c >= valid) s[c] = __float_as_uint(-INFINITY);
         }
-        const float mx = row_max<PAGE>(s);
+        const float mx_own = row_max<32>(s);
+        xch[grp * HQ + h] = mx_own;
+        // both groups have read S (its buffer may be refilled) and agree on the max
+        tc_fence_before();
+        good = named_bar_and(BAR_MAX, SOFTMAX_THREADS, good);
+        if (!good) { ok = false; break; }
+        if (threadIdx.x == 0) {
+          tc_fence_before();
+          mbar_arrive(bar(B_SB + (g & 1)));   // both groups have read this page's S
+        }
+        const float mx = fmaxf(mx_own, xch[(1 - grp) * HQ + h]);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = m_new > m_run + kRescaleThreshold;
         const float m_use = grow ? m_new : m_run;
         const float alpha = grow ? ex2(m_run - m_use) : 1.f;
         const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-        uint32_t p[PAGE / 2];
+        uint32_t p[16];
         // A page cut by the sequence end uses the MUFU exp2 only (its masked
         // scores are -inf and must give exactly 0); full pages send part of
         // the work to the FMA pipe.
-        const float sum = partial ? exp_row<PAGE, false>(s, p, sl2, m_eff) : exp_row<PAGE, true>(s, p, sl2, m_eff);
+        const float sum = partial ? exp_row<32, false>(s, p, sl2, m_eff) : exp_row<32, true>(s, p, sl2, m_eff);
         l_run = l_run * alpha + sum;
         m_run = m_use;
         if (gp > g0) {
           // the previous page's P V product must be complete before O changes
-          // (and before this page's P is announced: the P barrier then never
-          // runs two phases ahead of the P V issuer)
-          if (!warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          if (__any_sync(0xffffffffu, grow)) {
+          good = warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status);
+          if (good && __any_sync(0xffffffffu, grow)) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 256 / 32; ++c) {
+            for (int c = 0; c < 128 / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32_sync(t_row + O_COL + c * 32, o);
+              const uint32_t oc = t_row + O_COL + grp * 128 + c * 32;
+              tmem_ld32_sync(oc, o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(t_row + O_COL + c * 32, o);
+              tmem_st32(oc, o);
             }
           }
         }
-        tmem_st32(s_row, p);   // P over the first PAGE/2 columns of the S just read
-        tmem_st_wait();
+        // this group's 32 tokens of P into row h of the P tile (units 4G..4G+3
+        // of the 128-byte row, XOR-swizzled by h % 8 like a TMA tile)
+        {
+          const uint32_t prow = base + OFF_P + (uint32_t)h * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(prow + (((grp * 4 + k) ^ (h & 7)) * 16), p[4 * k], p[4 * k + 1], p[4 * k + 2], p[4 * k + 3]);
+          fence_proxy_async_smem();   // visible to the tensor core's reads
+        }
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_PF));
-      }
-      if (!ok) break;
-      // -------------------------------------------------------- segment epilogue
-      if (!warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
-      const bool full = (g0 == pref[sb]) && (g1 == pref[sb + 1]);
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      const float lse = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-      int slot = 2 * pair + (g0 == R0 ? 0 : 1);
-#pragma unroll 1
-      for (int c = 0; c < 256 / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32_sync(t_row + O_COL + c * 32, o);
-        const int col = half * 256 + c * 32;
-        if (full) {
-          uint4* dst = reinterpret_cast<uint4*>(a.o + ((size_t)sb * HQ + h) * DV + col);
+        good = named_bar_and(BAR_P, SOFTMAX_THREADS, good);
+        if (!good) { ok = false; break; }
+        if (warp == 0) {
+          // O (+)= P V for this page: P from TMEM, V = the own part (its slot
+          // is released by the same commit).  S of the page is complete, so
+          // its own part has landed.
+          tc_fence_after();
+          const bool leader = elect_one();
+          const int os = g % OWN_STAGES;
+          const uint64_t vdesc = sdesc_sw128(base + OFF_OWN + os * OWN_BYTES, PAGE_CHUNK_BYTES, 1024);
+          const uint64_t pdesc = sdesc_sw128(base + OFF_P, 16, 1024);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-            u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-            u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-            u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-            dst[i] = u;
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(a.ws_o + ((size_t)slot * HQ + h) * DV + col);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                 __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+          for (int kk = 0; kk < PAGE / 16; ++kk)
+            mma_ss(tmem + O_COL, pdesc + ((kk * 32) >> 4), vdesc + ((kk * 16 * 128) >> 4), idesc_o,
+                   (gp == g0 && kk == 0) ? 0u : 1u, leader);
+          mma_commit(bar(B_OD), leader);
+          mma_commit(bar(B_OE + os), leader);   // the own part's slot is free
+          __syncwarp();
         }
       }
-      if (half == 0) {
+      if (!ok) break;
+      // The next segment's Q goes into TMEM before this epilogue: the last
+      // score tile of this segment is complete (its softmax has run), so the
+      // next segment's first score tile can be computed during the epilogue.
+      int nsb = 0, ng0 = 0, ng1 = 0;
+      const bool nhave = w.next(nsb, ng0, ng1);
+      if (nhave) write_q_tmem(nsb);
+      // -------------------------------------------------------- segment epilogue
+      bool good = warp_wait(bar(B_OD), (g - 1) & 1, abort_flag, a.status);
+      tc_fence_after();
+      xch[grp * HQ + h] = l_run;
+      good = named_bar_and(BAR_L, SOFTMAX_THREADS, good);
+      if (!good) { ok = false; break; }
+      const float l_tot = l_run + xch[(1 - grp) * HQ + h];
+      const bool full = (g0 == pref[sb]) && (g1 == pref[sb + 1]);
+      const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      const float lse = (l_tot > 0.f) ? (m_run + log2f(l_tot)) * kLn2 : -INFINITY;
+      int slot = 2 * pair + (g0 == R0 ? 0 : 1);
+      // Each 32-column chunk of this warp's 32 rows goes through the warp's
+      // transpose tile (16-byte units XOR-swizzled by row, so neither side has
+      // bank conflicts); read back by rows, every store instruction then
+      // writes 4 rows x 128 bytes (fp32) or 8 rows x 64 bytes (bf16) instead
+      // of 32 rows x 16 bytes.
+      const uint32_t xt = base + OFF_XPOSE + (uint32_t)((grp * 4 + q4) * XPOSE_BYTES);
+      const int row0 = q4 * 32;   // first head of this warp
+#pragma unroll 1
+      for (int c = 0; c < 128 / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32_sync(t_row + O_COL + grp * 128 + c * 32, o);
+        const int col = half * 256 + grp * 128 + c * 32;
+        if (full) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(xt + lane * 128 + ((k ^ (lane & 7)) * 16),
+                         pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = 8 * j + (lane >> 2), u = lane & 3;
+            uint32_t v0, v1, v2, v3;
+            ld_shared_v4(xt + r * 128 + ((u ^ (r & 7)) * 16), v0, v1, v2, v3);
+            *reinterpret_cast<uint4*>(a.o + ((size_t)sb * HQ + row0 + r) * DV + col + 8 * u) = make_uint4(v0, v1, v2, v3);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(xt + lane * 128 + ((k ^ (lane & 7)) * 16),
+                         __float_as_uint(__uint_as_float(o[4 * k + 0]) * inv_l),
+                         __float_as_uint(__uint_as_float(o[4 * k + 1]) * inv_l),
+                         __float_as_uint(__uint_as_float(o[4 * k + 2]) * inv_l),
+                         __float_as_uint(__uint_as_float(o[4 * k + 3]) * inv_l));
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int r = 4 * j + (lane >> 3), u = lane & 7;
+            uint32_t v0, v1, v2, v3;
+            ld_shared_v4(xt + r * 128 + ((u ^ (r & 7)) * 16), v0, v1, v2, v3);
+            *reinterpret_cast<uint4*>(a.ws_o + ((size_t)slot * HQ + row0 + r) * DV + col + 4 * u) =
+                make_uint4(v0, v1, v2, v3);
+          }
+        }
+        __syncwarp();   // the tile is rewritten by the next chunk
+      }
+      if (half == 0 && grp == 0) {
         if (full) a.lse[(size_t)sb * HQ + h] = lse;
         else a.ws_lse[(size_t)slot * HQ + h] = lse;
       }
       tc_fence_before();
       __syncwarp();
       ++seg;
+      sb = nsb;
+      g0 = ng0;
+      g1 = ng1;
+      have = nhave;
+    }
+    if (warp == 0) {
+      // Drain: no P V product may still run when TMEM is released.
+      const bool leader = elect_one();
+      mma_commit(bar(B_DR), leader);
+      __syncwarp();
+      mbar_wait_drain(bar(B_DR), 0);
     }
     __syncwarp();
   }
@@ -616,6 +730,9 @@ constexpr int MAX_PARTS = 128;   // >= CTA pairs, so a sequence never has more p
 
 __global__ void __launch_bounds__(COMBINE_THREADS)
     decode_combine_kernel(const Args a) {
+  // Launched as a programmatic dependent of the split kernel: wait here until
+  // that grid has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int h0 = blockIdx.y * COMBINE_HEADS;
   const int tid = threadIdx.x;
@@ -659,21 +776,39 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
     a.lse[(size_t)b * HQ + h] = sum > 0.f ? mx + logf(sum) : -INFINITY;
   }
   __syncthreads();
-  // 16 heads x 512 columns, 4 columns per thread per step
-  for (int i = tid; i < COMBINE_HEADS * DV / 4; i += COMBINE_THREADS) {
-    const int hh = i / (DV / 4), c4 = i % (DV / 4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < nparts && j < MAX_PARTS; ++j) {
-      const float wgt = w_s[hh][j];
-      const float4 v = *reinterpret_cast<const float4*>(a.ws_o + ((size_t)slot_s[j] * HQ + h0 + hh) * DV + c4 * 4);
-      acc.x += wgt * v.x;
-      acc.y += wgt * v.y;
-      acc.z += wgt * v.z;
-      acc.w += wgt * v.w;
+  // 16 heads x 512 columns: each thread owns OUT_PER_THREAD groups of 4
+  // columns (head hh = tid / 128 + 2k, columns 4 (tid % 128) ..), and the
+  // loads of one piece for all of them are issued together, so a piece costs
+  // one memory latency rather than one per group.
+  constexpr int OUT_PER_THREAD = COMBINE_HEADS * DV / 4 / COMBINE_THREADS;
+  static_assert(OUT_PER_THREAD * COMBINE_THREADS * 4 == COMBINE_HEADS * DV && COMBINE_THREADS % (DV / 4) == 0,
+                "combine thread map");
+  const int c4 = tid % (DV / 4), hh0 = tid / (DV / 4);
+  constexpr int HH_STEP = COMBINE_THREADS / (DV / 4);
+  float4 acc[OUT_PER_THREAD];
+#pragma unroll
+  for (int k = 0; k < OUT_PER_THREAD; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < nparts && j < MAX_PARTS; ++j) {
+    const float* src = a.ws_o + ((size_t)slot_s[j] * HQ + h0) * DV + c4 * 4;
+    float4 v[OUT_PER_THREAD];
+#pragma unroll
+    for (int k = 0; k < OUT_PER_THREAD; ++k)
+      v[k] = *reinterpret_cast<const float4*>(src + (size_t)(hh0 + HH_STEP * k) * DV);
+#pragma unroll
+    for (int k = 0; k < OUT_PER_THREAD; ++k) {
+      const float wgt = w_s[hh0 + HH_STEP * k][j];
+      acc[k].x += wgt * v[k].x;
+      acc[k].y += wgt * v[k].y;
+      acc[k].z += wgt * v[k].z;
+      acc[k].w += wgt * v[k].w;
     }
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh) * DV + c4 * 4);
-    dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
-    dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+  }
+#pragma unroll
+  for (int k = 0; k < OUT_PER_THREAD; ++k) {
+    __nv_bfloat162* dst =
+        reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh0 + HH_STEP * k) * DV + c4 * 4);
+    dst[0] = __floats2bfloat162_rn(acc[k].x, acc[k].y);
+    dst[1] = __floats2bfloat162_rn(acc[k].z, acc[k].w);
   }
 }
 
@@ -773,7 +908,20 @@ extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   decode_split_kernel<<<2 * pairs, THREADS, SMEM_BYTES, s>>>(tq, tkv, a);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  decode_combine_kernel<<<dim3(units, HQ / COMBINE_HEADS), COMBINE_THREADS, 0, s>>>(a);
+  // The combine is a programmatic dependent launch: its CTAs are scheduled as
+  // the split kernel's CTAs retire and wait (griddepcontrol.wait) for that
+  // grid's completion, instead of the stream's full launch gap.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units, HQ / COMBINE_HEADS);
+  cfg.blockDim = dim3(COMBINE_THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, a) != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
