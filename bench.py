@@ -61,10 +61,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu capture of the same launch; see profiles/.  Set to None whenever the
 # kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 201555456 + 106562560,   # attn_fwd_kernel<D=128, causal>, GQA N=16384 workload
-    "decode": 349649664 + 16860928,     # decode_split_kernel, MLA decode workload
+    "prefill": 372582656 + 105771008,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
+    "prefill_c4": 152573952 + 101151488,   # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload
+    "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
-    "bwd": 2549769216 + 1224851200,     # attn_bwd_kernel<D=128, causal>, same workload (backward)
+    "bwd": 2360328704 + 1253101056,     # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
     "fp8": 100732160 + 92020992,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
 }
 # Timed regions longer than this run under the power cap: compare with the
@@ -498,7 +499,7 @@ def run_gpu(args):
         objs["fp8"] = o
     if "bwd" in by:
         o = tensor_obj(by["bwd"], "attention backward TFLOP/s",
-                       "bwd_prep_kernel + attn_bwd_kernel<D=128,causal> + bwd_dq_kernel (timed together)",
+                       "bwd_prep_kernel + attn_bwd_dqt_kernel<causal> + bwd_dqt_kernel (timed together)",
                        bf16_peak, bf16_kind, NCU_TRAFFIC_BYTES.get("bwd"))
         o["config"]["flops"] = "2.5 x forward (five products)"
         objs["bwd"] = o

@@ -172,6 +172,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   int* pref = reinterpret_cast<int*>(base_ptr + C::OFF_PREF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::OFF_MISC);
 
+  // Let the combine kernel be scheduled as this grid's CTAs retire (it waits
+  // for this grid's completion before reading anything).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pw = warp >> 1;     // worker = pair of warps
   const int half = warp & 1;    // this warp's tokens of every page: [32 half, 32 half + 32)
@@ -510,6 +513,9 @@ constexpr int COMBINE_CHUNK = 128;
 constexpr int COMBINE_OUT = 8;   // output elements per thread: G * D <= 8 * 128
 
 __global__ void __launch_bounds__(COMBINE_THREADS) gqa_combine_kernel(const Args a) {
+  // Launched as a programmatic dependent of the decode kernel: wait here until
+  // that grid has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x, g = blockIdx.y;
   const int G = a.G, D = a.D, Hq = a.Hkv * G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -728,6 +734,17 @@ extern "C" int attn_decode_paged_gqa(const void* q, const void* k_pages, const v
                 : launch<64, 8>(tk, tv, a, sms, s);
   }
   if (rc != ATTN_OK) return rc;
-  gqa_combine_kernel<<<dim3(B, Hkv), COMBINE_THREADS, 0, s>>>(a);
+  // a programmatic dependent launch, like the MLA decode's combine
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B, Hkv);
+  cfg.blockDim = dim3(COMBINE_THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gqa_combine_kernel, a) != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -3,9 +3,12 @@
 // What it computes ("FlashAttention (KO)": the attention formula, tiling,
 // online softmax, fusion into one kernel):
 //   O = softmax(scale * Q K^T + causal mask) V, LSE = ln sum exp(scale * Q K^T)
-// without writing S to device memory.  Each CTA owns NT query tiles of 128
-// rows of one (batch, query head) and streams the KV head's K/V in blocks of
-// BN keys through shared memory:
+// without writing S to device memory.  The kernel is persistent: one CTA per
+// SM walks work units (NT query tiles of 128 rows of one (batch, query head))
+// in a static snake order over a list ordered heaviest first, keeping its
+// tensor memory, barriers and rings across units, so one unit's loads and
+// first score tile overlap the previous unit's epilogue.  Per unit it streams the
+// KV head's K/V in blocks of BN keys through shared memory:
 //
 //   producer warp   TMA: Q tiles once, then a ring of K and V blocks
 //   MMA warp        one thread issues tcgen05.mma:  S = Q K^T  into TMEM,
@@ -29,6 +32,8 @@
 // folded into the score scale and the V descale into the epilogue.
 #include <math.h>
 
+#include <algorithm>
+
 #include "host_common.h"
 #include "sm100.cuh"
 #include "softmax_row.cuh"
@@ -51,8 +56,11 @@ struct FwdCfg {
   static constexpr int NSL = (NT == 1 || 2 * BN + D <= 256) ? 2 : 1;
   static constexpr int KV_TILE = BN * D * ES;
   // FP8 stages the bf16 O tiles in a region of their own (the e4m3 Q tile is
-  // half their size); bf16 reuses the dead Q tile.
-  static constexpr int O_STAGE_BYTES = FP8 ? NT * 128 * D * 2 : 0;
+  // half their size), and so does head dim 64, whose rings have room to
+  // spare: the next unit's Q tiles can then be loaded while this unit's O is
+  // stored.  Head dims 128 and 256 stage O in the dead Q tile.
+  static constexpr bool SEP_OSTAGE = FP8 || D == 64;
+  static constexpr int O_STAGE_BYTES = SEP_OSTAGE ? NT * 128 * D * 2 : 0;
   static constexpr int KV_BUDGET = 224 * 1024 - NT * BM * D * ES - O_STAGE_BYTES;   // shared memory left for K/V
   static constexpr int KSTAGES = (KV_BUDGET / KV_TILE + 1) / 2;      // K ring (released after S)
   static constexpr int VSTAGES = KV_BUDGET / KV_TILE - KSTAGES;      // V ring (held until P V)
@@ -71,11 +79,12 @@ struct FwdCfg {
   static constexpr float RESCALE_THR = FP8 ? 4.0f : 8.0f;
   static constexpr float P_SHIFT = FP8 ? 4.0f : 0.0f;
   static constexpr int SOFTMAX_WARPS = 4 * NT;
-  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // Q and K loads
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // K loads
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
   static constexpr int V_PRODUCER_WARP = SOFTMAX_WARPS + 2;  // V loads, never queued behind K
-  // The three issuing warps plus one idle warp form a full warpgroup, so the
-  // register budget can move from it to the softmax warpgroups.
+  static constexpr int Q_PRODUCER_WARP = SOFTMAX_WARPS + 3;  // Q tiles, which wait for the previous epilogue
+  // The four issuing warps form a full warpgroup, so the register budget can
+  // move from it to the softmax warpgroups.
   static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
   static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
   static constexpr int ISSUE_REGS = 56;
@@ -100,8 +109,13 @@ struct FwdCfg {
   // issued after P_j V_j), so no barrier ever runs two phases ahead.
   static constexpr int B_PF = B_SF + NT * NSL;
   static constexpr int B_OD = B_PF + NT * NSL;      // one phase per P V product of the tile
-  static constexpr int B_OF = B_OD + NT;      // single phase: the tile's last P V is done
-  static constexpr int B_DR = B_OF + NT;
+  static constexpr int B_OF = B_OD + NT;      // one phase per unit: the tile's last P V is done
+  // Q tile t may be reloaded: its staging of O has been read by the TMA store
+  // (O staged in the Q tile), or its unit's last score tile is done (O staged
+  // apart).  One phase per unit that arrives on it.
+  static constexpr int B_QE = B_OF + NT;
+  static constexpr int B_OR = B_QE + NT;      // the epilogue has read O of tile t from TMEM (4 warps)
+  static constexpr int B_DR = B_OR + NT;
   static constexpr int NBAR = B_DR + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_Q = 0;
@@ -120,10 +134,36 @@ struct FwdCfg {
 struct FwdArgs {
   float* lse;
   int* status;
-  int Hq, Nq, Nk, group, n_qblk, causal_off;
+  int B, Hq, Nq, Nk, group, n_qblk, causal_off;
+  int n_units;        // n_qblk * Hq * B work units
   float scale_log2;   // scale * log2(e) (FP8: times the Q and K descales)
   float o_mul;        // 1 (FP8: the V descale)
 };
+
+// Work unit u: query-block index slowest (heaviest first under the causal
+// mask), then query head (heads of one KV group adjacent, so their K/V are
+// read from L2), then batch.
+struct Unit {
+  int qblk, hq, b;
+};
+
+// The k-th unit of CTA `cta` in a grid of `grid` CTAs: a static snake order
+// over the heaviest-first list (rounds of `grid` units, every other round
+// taken backwards), so that under the causal mask each CTA's total work is
+// even.  Returns -1 past the last unit.
+__device__ __forceinline__ int unit_index(int cta, int grid, int k, int n_units) {
+  const long long u = (long long)k * grid + ((k & 1) ? (grid - 1 - cta) : cta);
+  return u < n_units ? (int)u : -1;
+}
+__device__ __forceinline__ Unit unit_of(const FwdArgs& a, int u, bool causal) {
+  const int per = a.Hq * a.B;
+  const int qi = u / per, r = u - qi * per;
+  Unit x;
+  x.qblk = causal ? (a.n_qblk - 1 - qi) : qi;
+  x.hq = r % a.Hq;
+  x.b = r / a.Hq;
+  return x;
+}
 
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -142,32 +182,43 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qblk = C::CAUSAL ? (a.n_qblk - 1 - (int)blockIdx.x) : (int)blockIdx.x;   // heaviest first
-  const int hq = blockIdx.y, b = blockIdx.z;
-  const int hk = hq / a.group;
 
-  // Number of key blocks each tile visits.
-  int nblk[NT];
-  int nmax = 0;
+  // Key blocks each tile of unit x visits (0 for a tile past Nq, or one whose
+  // rows see no key); returns the most over the tiles.
+  auto unit_blocks = [&](const Unit& x, int* nblk) -> int {
+    int nmax = 0;
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int r0 = (qblk * NT + t) * C::BM;
-    int n = 0;
-    if (r0 < a.Nq) {
-      int kv_end = a.Nk;
-      if (C::CAUSAL) {
-        const int last_row = min(r0 + C::BM, a.Nq) - 1;
-        kv_end = min(a.Nk, last_row + a.causal_off + 1);
+    for (int t = 0; t < NT; ++t) {
+      const int r0 = (x.qblk * NT + t) * C::BM;
+      int n = 0;
+      if (r0 < a.Nq) {
+        int kv_end = a.Nk;
+        if (C::CAUSAL) {
+          const int last_row = min(r0 + C::BM, a.Nq) - 1;
+          kv_end = min(a.Nk, last_row + a.causal_off + 1);
+        }
+        n = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;
       }
-      n = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;
+      nblk[t] = n;
+      nmax = max(nmax, n);
     }
-    nblk[t] = n;
-    nmax = max(nmax, n);
-  }
+    return nmax;
+  };
+  // A tile is active in unit x when it holds rows below Nq: its epilogue
+  // writes O and LSE (zeros and -inf if it saw no key).
+  auto tile_active = [&](const Unit& x, int t) { return (x.qblk * NT + t) * C::BM < a.Nq; };
+  // Arrivals unit x brings on the Q-free barrier of tile t.
+  auto qe_arrivals = [&](const Unit& x, const int* nblk, int t) -> int {
+    return C::SEP_OSTAGE ? (nblk[t] > 0 ? 1 : 0) : (tile_active(x, t) ? 1 : 0);
+  };
 
   if (threadIdx.x == 0) {
 #pragma unroll
-    for (int t = 0; t < NT; ++t) mbar_init(bar(C::B_QF + t), 1);
+    for (int t = 0; t < NT; ++t) {
+      mbar_init(bar(C::B_QF + t), 1);
+      mbar_init(bar(C::B_QE + t), 1);
+      mbar_init(bar(C::B_OR + t), 4);   // one arrival per softmax warp of the tile
+    }
 #pragma unroll
     for (int s = 0; s < KST; ++s) {
       mbar_init(bar(C::B_KF + s), 1);
@@ -210,127 +261,196 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ============================================================ issue warpgroup
     if constexpr (C::NT == 2) regs_decrease<C::ISSUE_REGS>();
   if (warp == C::PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ K producer
+    // K blocks of every unit through the K ring; never waits on an epilogue,
+    // so the next unit's first blocks are loaded while this unit finishes.
     if (lane == 0) {
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        if (nblk[t] > 0) {
-          const int r0 = (qblk * NT + t) * C::BM;
-          mbar_arrive_expect_tx(bar(C::B_QF + t), C::Q_BYTES);
+      int kc = 0;   // K blocks issued so far (ring slot and phase)
+      bool ok = true;
+      for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+        const Unit x = unit_of(a, u, C::CAUSAL);
+        int nblk[NT];
+        const int nmax = unit_blocks(x, nblk);
+        const int hk = x.hq / a.group;
+        for (int j = 0; j < nmax; ++j, ++kc) {
+          const int st = kc % KST;
+          if (!mbar_wait(bar(C::B_KE + st), ((kc / KST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_4d(base + C::OFF_Q + t * C::Q_BYTES + ch * C::Q_CHUNK, &tm_q, bar(C::B_QF + t),
-                        ch * C::CH_ELEMS, hq, r0, b);
+            tma_load_4d(base + C::OFF_K + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_k, bar(C::B_KF + st),
+                        ch * C::CH_ELEMS, hk, j * BN, x.b);
         }
       }
-      int k_issued = 0;
-      for (int j = 0; j < nmax; ++j) {
-        const int st = j % KST;
-        if (!mbar_wait(bar(C::B_KE + st), ((j / KST) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(bar(C::B_KF + st), C::KV_BYTES);
-#pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_4d(base + C::OFF_K + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_k, bar(C::B_KF + st),
-                      ch * C::CH_ELEMS, hk, j * BN, b);
-        ++k_issued;
-      }
       // Drain: every issued copy must land before shared memory is released.
-      for (int j = max(0, k_issued - KST); j < k_issued; ++j) mbar_wait_drain(bar(C::B_KF + j % KST), (j / KST) & 1);
-#pragma unroll
-      for (int t = 0; t < NT; ++t)
-        if (nblk[t] > 0) mbar_wait_drain(bar(C::B_QF + t), 0);
+      for (int j = max(0, kc - KST); j < kc; ++j) mbar_wait_drain(bar(C::B_KF + j % KST), (j / KST) & 1);
     }
     __syncwarp();
   } else if (warp == C::V_PRODUCER_WARP) {
     // ------------------------------------------------------------ V producer
     if (lane == 0) {
-      int v_issued = 0;
-      for (int j = 0; j < nmax; ++j) {
-        const int st = j % VST;
-        if (!mbar_wait(bar(C::B_VE + st), ((j / VST) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(bar(C::B_VF + st), C::KV_BYTES);
+      int vc = 0;
+      bool ok = true;
+      for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+        const Unit x = unit_of(a, u, C::CAUSAL);
+        int nblk[NT];
+        const int nmax = unit_blocks(x, nblk);
+        const int hk = x.hq / a.group;
+        for (int j = 0; j < nmax; ++j, ++vc) {
+          const int st = vc % VST;
+          if (!mbar_wait(bar(C::B_VE + st), ((vc / VST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(C::B_VF + st), C::KV_BYTES);
 #pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_4d(base + C::OFF_V + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_v, bar(C::B_VF + st),
-                      ch * C::CH_ELEMS, hk, j * BN, b);
-        ++v_issued;
+          for (int ch = 0; ch < C::DCH; ++ch)
+            tma_load_4d(base + C::OFF_V + st * C::KV_BYTES + ch * C::KV_CHUNK, &tm_v, bar(C::B_VF + st),
+                        ch * C::CH_ELEMS, hk, j * BN, x.b);
+        }
       }
-      for (int j = max(0, v_issued - VST); j < v_issued; ++j) mbar_wait_drain(bar(C::B_VF + j % VST), (j / VST) & 1);
+      for (int j = max(0, vc - VST); j < vc; ++j) mbar_wait_drain(bar(C::B_VF + j % VST), (j / VST) & 1);
+    }
+    __syncwarp();
+  } else if (warp == C::Q_PRODUCER_WARP) {
+    // ------------------------------------------------------------ Q producer
+    // Q tile t of a unit is loaded once the tile's buffer is free again: its
+    // O staging has been read by the previous epilogue's TMA store (O staged
+    // in the Q tile) or the previous unit's last score tile is done.
+    if (lane == 0) {
+      int qld[NT] = {};   // Q loads issued per tile
+      int qe[NT] = {};    // arrivals earlier units bring on the tile's Q-free barrier
+      bool ok = true;
+      for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+        const Unit x = unit_of(a, u, C::CAUSAL);
+        int nblk[NT];
+        unit_blocks(x, nblk);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (!ok) break;
+          if (nblk[t] > 0) {
+            // the latest earlier arrival is the last one: a later unit's cannot
+            // come before this load (it needs this Q, or has no Q tile to wait for)
+            if (qe[t] > 0 && !mbar_wait(bar(C::B_QE + t), (qe[t] - 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            const int r0 = (x.qblk * NT + t) * C::BM;
+            mbar_arrive_expect_tx(bar(C::B_QF + t), C::Q_BYTES);
+#pragma unroll
+            for (int ch = 0; ch < C::DCH; ++ch)
+              tma_load_4d(base + C::OFF_Q + t * C::Q_BYTES + ch * C::Q_CHUNK, &tm_q, bar(C::B_QF + t),
+                          ch * C::CH_ELEMS, x.hq, r0, x.b);
+            ++qld[t];
+          }
+          qe[t] += qe_arrivals(x, nblk, t);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        if (qld[t] > 0) mbar_wait_drain(bar(C::B_QF + t), (qld[t] - 1) & 1);
     }
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the schedule (descriptors stay warp-uniform); one
     // elected lane issues each tcgen05 instruction, predicated (no branch).
+    // Ring slots, S buffers and barrier phases are indexed by running counts
+    // over the units, so they carry across units unchanged.
     const bool leader = elect_one();
     constexpr uint32_t idesc_s = C::FP8 ? idesc_e4m3_f32(128, BN, false) : idesc_bf16_f32(128, BN, false);
     constexpr uint32_t idesc_o = C::FP8 ? idesc_e4m3_f32(128, D, true) : idesc_bf16_f32(128, D, true);
+    int kc = 0, vc = 0;   // K and V blocks consumed before this unit
+    int sc[NT] = {};      // score tiles of tile t before this unit
+    int qld[NT] = {};     // Q loads of tile t consumed
+    int orc[NT] = {};     // epilogues of tile t before this unit (arrivals on its O-read barrier)
     bool ok = true;
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-      if (ok && nblk[t] > 0) ok = warp_wait(bar(C::B_QF + t), 0, abort_flag, a.status);
-
-    auto last_tile = [&](int j) {
-      int lt = -1;
+    for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+      const Unit x = unit_of(a, u, C::CAUSAL);
+      int nblk[NT];
+      const int nmax = unit_blocks(x, nblk);
 #pragma unroll
       for (int t = 0; t < NT; ++t)
-        if (j < nblk[t]) lt = t;
-      return lt;
-    };
-    // S(t, j) = Q_t K_j^T into S buffer j % NSL of tile t.
-    auto issue_s = [&](int t, int j) -> bool {
-      const int st = j % KST;
-      if (!warp_wait(bar(C::B_KF + st), (j / KST) & 1, abort_flag, a.status)) return false;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
-      const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
-      const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
+        if (ok && nblk[t] > 0) {
+          ok = warp_wait(bar(C::B_QF + t), qld[t] & 1, abort_flag, a.status);
+          ++qld[t];
+        }
+
+      auto last_tile = [&](int j) {
+        int lt = -1;
 #pragma unroll
-      for (int ks = 0; ks < D / C::K_MMA; ++ks) {
-        // advance the start-address field (16-byte units) to k-step ks (32 bytes of a row)
-        const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
-        const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
-        if constexpr (C::FP8) mma_ss_f8(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
-        else mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+        for (int t = 0; t < NT; ++t)
+          if (j < nblk[t]) lt = t;
+        return lt;
+      };
+      // S(t, j) = Q_t K_j^T into S buffer (sc[t] + j) % NSL of tile t.
+      auto issue_s = [&](int t, int j) -> bool {
+        const int kj = kc + j, st = kj % KST;
+        if (!warp_wait(bar(C::B_KF + st), (kj / KST) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const int c = sc[t] + j;
+        const uint32_t d_tmem = tmem + t * C::TILE_COLS + (c % NSL) * BN;
+        const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
+        const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < D / C::K_MMA; ++ks) {
+          // advance the start-address field (16-byte units) to k-step ks (32 bytes of a row)
+          const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
+          const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
+          if constexpr (C::FP8) mma_ss_f8(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+          else mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+        }
+        mma_commit(bar(C::B_SF + t * NSL + (c % NSL)), leader);
+        if (t == last_tile(j)) mma_commit(bar(C::B_KE + st), leader);
+        // O staged apart: the Q tile is free once the unit's last score tile is done
+        if (C::SEP_OSTAGE && j == nblk[t] - 1) mma_commit(bar(C::B_QE + t), leader);
+        __syncwarp();
+        return true;
+      };
+
+      for (int i = 0; ok && i < NSL; ++i)
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          if (ok && i < nblk[t]) ok = issue_s(t, i);
+
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int vj = vc + j, st = vj % VST;
+        bool v_ready = false;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (!ok || j >= nblk[t]) continue;
+          const int c = sc[t] + j;
+          if (!warp_wait(bar(C::B_PF + t * NSL + c % NSL), (c / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!v_ready) {
+            if (!warp_wait(bar(C::B_VF + st), (vj / VST) & 1, abort_flag, a.status)) { ok = false; break; }
+            v_ready = true;
+          }
+          // The unit's first product overwrites O: the previous epilogue of
+          // this tile must have read it (its latest arrival is the last one,
+          // since the next epilogue needs this unit's products).
+          if (j == 0 && orc[t] > 0 &&
+              !warp_wait(bar(C::B_OR + t), (orc[t] - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t p_tmem = tmem + t * C::TILE_COLS + (c % NSL) * BN;
+          const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
+          const uint64_t vdesc = sdesc_sw128(base + C::OFF_V + st * C::KV_BYTES, C::KV_CHUNK, 1024);
+#pragma unroll
+          for (int ks = 0; ks < BN / C::K_MMA; ++ks) {
+            // K_MMA keys per step: 8 TMEM columns of packed P, K_MMA rows of V
+            const uint64_t vd = vdesc + ((ks * C::K_MMA * 128) >> 4);
+            if constexpr (C::FP8) mma_ts_f8(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
+            else mma_ts(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
+          }
+          mma_commit(bar(C::B_OD + t), leader);
+          if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t), leader);
+          if (t == last_tile(j)) mma_commit(bar(C::B_VE + st), leader);
+          __syncwarp();
+          if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
+        }
       }
-      mma_commit(bar(C::B_SF + t * NSL + (j % NSL)), leader);
-      if (t == last_tile(j)) mma_commit(bar(C::B_KE + st), leader);
-      __syncwarp();
-      return true;
-    };
-
-    for (int i = 0; ok && i < NSL; ++i)
-#pragma unroll
-      for (int t = 0; t < NT; ++t)
-        if (ok && i < nblk[t]) ok = issue_s(t, i);
-
-    for (int j = 0; ok && j < nmax; ++j) {
-      const int st = j % VST;
-      bool v_ready = false;
+      kc += nmax;
+      vc += nmax;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        if (!ok || j >= nblk[t]) continue;
-        if (!warp_wait(bar(C::B_PF + t * NSL + j % NSL), (j / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
-        if (!v_ready) {
-          if (!warp_wait(bar(C::B_VF + st), (j / VST) & 1, abort_flag, a.status)) { ok = false; break; }
-          v_ready = true;
-        }
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + t * C::TILE_COLS + (j % NSL) * BN;
-        const uint32_t o_tmem = tmem + t * C::TILE_COLS + C::O_COL;
-        const uint64_t vdesc = sdesc_sw128(base + C::OFF_V + st * C::KV_BYTES, C::KV_CHUNK, 1024);
-#pragma unroll
-        for (int ks = 0; ks < BN / C::K_MMA; ++ks) {
-          // K_MMA keys per step: 8 TMEM columns of packed P, K_MMA rows of V
-          const uint64_t vd = vdesc + ((ks * C::K_MMA * 128) >> 4);
-          if constexpr (C::FP8) mma_ts_f8(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
-          else mma_ts(o_tmem, p_tmem + ks * 8, vd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u, leader);
-        }
-        mma_commit(bar(C::B_OD + t), leader);
-        if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t), leader);
-        if (t == last_tile(j)) mma_commit(bar(C::B_VE + st), leader);
-        __syncwarp();
-        if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
+        sc[t] += nblk[t];
+        orc[t] += tile_active(x, t) ? 1 : 0;
       }
     }
     // Drain: no MMA may still run when TMEM is released.
@@ -345,119 +465,143 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int row_in_tile = wq * 32 + lane;
-    const int r0 = (qblk * NT + t) * C::BM;
-    const int row = r0 + row_in_tile;
-    const int n = nblk[t];
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t t_tmem = tmem + t * C::TILE_COLS + lane_off;
-    int lim = a.Nk;   // keys kk < lim are visible to this row
-    if (C::CAUSAL) lim = min(a.Nk, row + a.causal_off + 1);
     const float sl2 = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    int sc = 0;    // score tiles of this tile before the current unit
+    int ofc = 0;   // phases of this tile's last-product barrier consumed
     bool ok = true;
+    for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+      const Unit x = unit_of(a, u, C::CAUSAL);
+      int nblk[NT];
+      unit_blocks(x, nblk);
+      const int n = nblk[t];
+      const int r0 = (x.qblk * NT + t) * C::BM;
+      const int row = r0 + row_in_tile;
+      int lim = a.Nk;   // keys kk < lim are visible to this row
+      if (C::CAUSAL) lim = min(a.Nk, row + a.causal_off + 1);
+      float m_run = -INFINITY, l_run = 0.f;
 
-    for (int j = 0; j < n; ++j) {
-      const int slot = j % NSL;
-      if (!warp_wait(bar(C::B_SF + t * NSL + slot), (j / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s[BN];
-if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
-      else tmem_ld64_sync(t_tmem + slot * BN, s);
-
-      const bool need_mask = ((j + 1) * BN > a.Nk) || (C::CAUSAL && (j + 1) * BN - 1 > r0 + a.causal_off);
-      if (need_mask) {
-        const int cl = lim - j * BN;
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c >= cl) s[c] = __float_as_uint(-INFINITY);
-      }
-      const float mx = row_max<BN>(s);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const bool grow = m_new > m_run + C::RESCALE_THR;
-      const float m_use = grow ? m_new : m_run;
-      const float alpha = grow ? ex2(m_run - m_use) : 1.f;
-      // p is measured from 2^P_SHIFT below the reference max (l and O carry
-      // the same factor, so O/l is unchanged; the LSE subtracts it again)
-      const float m_eff = ((m_use == -INFINITY) ? 0.f : m_use) - C::P_SHIFT;
-      uint32_t p[C::P_WORDS];
-      // Blocks with masked keys use the MUFU exp2 only (masked scores are -inf
-      // and must give exactly 0); full blocks send part of the work to the FMA pipe.
-      float sum;
-      if constexpr (C::FP8)
-        sum = need_mask ? exp_row_e4m3<BN, false>(s, p, sl2, m_eff) : exp_row_e4m3<BN, true>(s, p, sl2, m_eff);
-      else
-        sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
-      l_run = l_run * alpha + sum;
-      m_run = m_use;
-#pragma unroll
-      for (int c = 0; c < C::P_WORDS / 32; ++c) tmem_st32(t_tmem + slot * BN + c * 32, p + c * 32);
-      tmem_st_wait();
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled.  The wait is
-        // unambiguous although most phases of this barrier are never waited
-        // on: S_j is done, so every P V issued before it (up to P_{j-2} V_{j-2})
-        // is done, and P_j V_j cannot start before this warp's arrival below;
-        // the barrier therefore sits at phase j-1 or j.
-        if (!warp_wait(bar(C::B_OD + t), (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      for (int j = 0; j < n; ++j) {
+        const int c = sc + j;
+        const int slot = c % NSL;
+        if (!warp_wait(bar(C::B_SF + t * NSL + slot), (c / NSL) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_tmem + C::O_COL + c * 32, o);
-        }
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PF + t * NSL + slot));
-    }
+        uint32_t s[BN];
+        if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
+        else tmem_ld64_sync(t_tmem + slot * BN, s);
 
-    // ------------------------------------------------------------ epilogue
-    if (ok && n > 0) {
-      ok = warp_wait(bar(C::B_OF + t), 0, abort_flag, a.status);
-      tc_fence_after();
-    }
-    const bool write = ok && !*abort_flag;
-    // bf16 O staging: the dead Q tile, or (FP8, whose Q tile is smaller) a region of its own
-    const uint32_t stage = C::FP8 ? base + C::OFF_OST + t * (128 * D * 2) : base + C::OFF_Q + t * C::Q_BYTES;
-    if (write) {
+        const bool need_mask = ((j + 1) * BN > a.Nk) || (C::CAUSAL && (j + 1) * BN - 1 > r0 + a.causal_off);
+        if (need_mask) {
+          const int cl = lim - j * BN;
+#pragma unroll
+          for (int cc = 0; cc < BN; ++cc)
+            if (cc >= cl) s[cc] = __float_as_uint(-INFINITY);
+        }
+        const float mx = row_max<BN>(s);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool grow = m_new > m_run + C::RESCALE_THR;
+        const float m_use = grow ? m_new : m_run;
+        const float alpha = grow ? ex2(m_run - m_use) : 1.f;
+        // p is measured from 2^P_SHIFT below the reference max (l and O carry
+        // the same factor, so O/l is unchanged; the LSE subtracts it again)
+        const float m_eff = ((m_use == -INFINITY) ? 0.f : m_use) - C::P_SHIFT;
+        uint32_t p[C::P_WORDS];
+        // Blocks with masked keys use the MUFU exp2 only (masked scores are -inf
+        // and must give exactly 0); full blocks send part of the work to the FMA pipe.
+        float sum;
+        if constexpr (C::FP8)
+          sum = need_mask ? exp_row_e4m3<BN, false>(s, p, sl2, m_eff) : exp_row_e4m3<BN, true>(s, p, sl2, m_eff);
+        else
+          sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
+        static_assert(C::P_WORDS % 32 == 0, "P rows are stored 32 columns at a time");
+#pragma unroll
+        for (int cc = 0; cc < C::P_WORDS / 32; ++cc) tmem_st32(t_tmem + slot * BN + cc * 32, p + cc * 32);
+        tmem_st_wait();
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O must hold P_{j-1} V_{j-1} before it is rescaled.  The wait is
+          // unambiguous although most phases of this barrier are never waited
+          // on: S_j is done, so every P V issued before it (up to P_{j-2} V_{j-2})
+          // is done, and P_j V_j cannot start before this warp's arrival below;
+          // the barrier therefore sits at phase c-1 or c (c = running index of S_j).
+          if (!warp_wait(bar(C::B_OD + t), (c - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_sync(t_tmem + C::O_COL + cc * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_tmem + C::O_COL + cc * 32, o);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_PF + t * NSL + slot));
+      }
+      sc += n;
+
+      // ------------------------------------------------------------ epilogue
+      if (!tile_active(x, t)) continue;
+      if (ok && n > 0) {
+        ok = warp_wait(bar(C::B_OF + t), ofc & 1, abort_flag, a.status);
+        tc_fence_after();
+      }
+      if (n > 0) ++ofc;
+      // The four warps of the tile take the same path from here on (a warp
+      // whose wait failed must not leave the others at a named barrier); the
+      // barrier also orders this staging after the previous unit's TMA store
+      // of the same area, which its issuing thread waited for before arriving.
+      ok = named_bar_and(1 + t, 128, ok && !*abort_flag);
+      const bool write = ok;
+      // bf16 O staging: the dead Q tile, or a region of its own
+      const uint32_t stage = C::SEP_OSTAGE ? base + C::OFF_OST + t * (128 * D * 2) : base + C::OFF_Q + t * C::Q_BYTES;
       const float inv_l = (l_run > 0.f) ? a.o_mul / l_run : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        if (n > 0) {
-          tmem_ld32_sync(t_tmem + C::O_COL + c * 32, o);
+        if (write && n > 0) {
+          tmem_ld32_sync(t_tmem + C::O_COL + cc * 32, o);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        uint32_t pk[16];
+        if (write) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        const uint32_t chunk = stage + (c >> 1) * C::Q_CHUNK + row_in_tile * 128;
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          const uint32_t chunk = stage + (cc >> 1) * C::Q_CHUNK + row_in_tile * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t unit = ((c & 1) * 4 + i) ^ (row_in_tile & 7);
-          st_shared_v4(chunk + unit * 16, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t unit = ((cc & 1) * 4 + i) ^ (row_in_tile & 7);
+            st_shared_v4(chunk + unit * 16, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
       }
-      fence_proxy_async_smem();
-    }
-    named_bar_sync(1 + t, 128);
-    if (write && wq == 0 && lane == 0 && r0 < a.Nq) {
+      // O of this tile has been read: the next unit's first product may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_OR + t));
+      if (write) fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (wq == 0 && lane == 0) {
+        if (write) {
 #pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) tma_store_4d(&tm_o, stage + ch * C::Q_CHUNK, ch * 64, hq, r0, b);   // bf16 O
-      tma_store_commit();
-      tma_store_wait_read();
+          for (int ch = 0; ch < D / 64; ++ch) tma_store_4d(&tm_o, stage + ch * C::Q_CHUNK, ch * 64, x.hq, r0, x.b);   // bf16 O
+          tma_store_commit();
+          tma_store_wait_read();
+        }
+        if (!C::SEP_OSTAGE) mbar_arrive(bar(C::B_QE + t));   // the Q tile may be reloaded
+      }
+      if (write && row < a.Nq)
+        a.lse[((size_t)x.b * a.Hq + x.hq) * a.Nq + row] =
+            (l_run > 0.f) ? (m_run - C::P_SHIFT + log2f(l_run)) * kLn2 : -INFINITY;
+      __syncwarp();
     }
-    if (write && row < a.Nq)
-      a.lse[((size_t)b * a.Hq + hq) * a.Nq + row] =
-          (l_run > 0.f) ? (m_run - C::P_SHIFT + log2f(l_run)) * kLn2 : -INFINITY;
-    __syncwarp();
   }
 
   tc_fence_before();
@@ -471,6 +615,10 @@ if constexpr (BN == 128) tmem_ld128_sync(t_tmem + slot * BN, s);
 template <int D, bool CAUSAL, bool FP8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                int Nk, float scale, cudaStream_t stream, float qk_descale = 1.f, float v_descale = 1.f) {
+  // 128-key blocks for head dims 64 and 128 (64-key blocks with two score
+  // buffers per tile measured slower there: 1169 against 1299 TFLOP/s for
+  // FP8, no change for head dim 64), 64-key blocks for head dim 256, whose
+  // single tile then fits two score buffers next to its 256-column O.
   using C = FwdCfg<D, CAUSAL, (D <= 128) ? 128 : 64, FP8>;
   static int attr_done = 0;
   const void* kfn = reinterpret_cast<const void*>(&attn_fwd_kernel<C>);
@@ -513,10 +661,18 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.Nk = Nk;
   a.group = Hq / Hkv;
   a.n_qblk = (Nq + C::BM * C::NT - 1) / (C::BM * C::NT);
+  a.B = B;
+  const long long units = (long long)a.n_qblk * Hq * B;
+  if (units >= (1ll << 31)) return ATTN_ERR_UNSUPPORTED;
+  a.n_units = (int)units;
   a.causal_off = Nk - Nq;
   a.scale_log2 = scale * qk_descale * 1.4426950408889634f;
   a.o_mul = v_descale;
-  dim3 grid(a.n_qblk, Hq, B);
+  // Persistent: one CTA per SM (the shared memory allows no more), each
+  // walking its units in the snake order.
+  const int sms = current_sm_count();
+  if (sms < 1) return ATTN_ERR_CUDA;
+  const int grid = (int)std::min<long long>(units, sms);
   attn_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

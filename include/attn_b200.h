@@ -236,8 +236,8 @@ int attn_decode_paged_mtp(const void* q, const void* kv_pages, const int32_t* bl
  * (attn_decode_paged_workspace_size) exceeds it is rejected with
  * ATTN_ERR_UNSUPPORTED before anything is enqueued.  The workspace grows with
  * the device's SM count; on a 148-SM B200 every batch up to the decode's
- * limit of 2048 sequences fits, so there only that limit applies.  The call allocates no
- * device memory.  The first call on each device looks up the array's device
+ * limit of 2048 sequences fits, so there only that limit applies.  The call
+ * allocates no device memory.  The first call on each device looks up the array's device
  * address (with that device current), so make it before any stream capture.
  * All calls share the array and it keeps the last call's contents: calls whose
  * kernels overlap on the GPU (several streams or threads) race on it and must

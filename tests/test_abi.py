@@ -131,6 +131,10 @@ def test_bwd_argument_checks(lib):
     assert call(Nq=0, Nk=0, q=None, dk=None, ws=None, wsb=0) == 0
     need = lib.attn_bwd_workspace_size(1, 4, 100, 128)
     assert need >= 100 * 4 * 128 * 4 + 100 * 4 * 4
+    # D = 128 keeps dQ transposed, each head dim's row of queries padded to a
+    # multiple of 32 (128 bytes) for the TMA adds: 100 -> 128 queries
+    assert need == 4 * 128 * 128 * 4 + 1792
+    assert lib.attn_bwd_workspace_size(1, 4, 100, 64) == 100 * 4 * 64 * 4 + 1792
     assert lib.attn_bwd_workspace_size(1, 4, 100, 256) == 0
 
 

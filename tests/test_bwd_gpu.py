@@ -90,14 +90,18 @@ def test_unequal_lengths(Nq, Nk, causal):
     _check(1, 4, 1, Nq, Nk, 128, causal, seed=Nq * 3 + Nk)
 
 
-def test_many_query_blocks_per_key_block():
-    """A long non-causal case: each CTA walks 16 query blocks x 2 heads."""
-    _check(1, 4, 2, 2048, 256, 64, False, seed=31)
+@pytest.mark.parametrize("D,Nq", [(64, 2048), (128, 2000)])
+def test_many_query_blocks_per_key_block(D, Nq):
+    """A long non-causal case: each CTA walks 16 (D = 64) or 32 (D = 128)
+    query blocks x 2 heads; 2000 queries leave a ragged last block and a
+    padded accumulator row."""
+    _check(1, 4, 2, Nq, 256, D, False, seed=31 + D)
 
 
-def test_empty_query_or_key_side():
+@pytest.mark.parametrize("D", [64, 128])
+def test_empty_query_or_key_side(D):
     d = torch.device("cuda:0")
-    q, k, v, do = inputs.bwd_inputs(1, 2, 1, 0, 130, 64, 3)
+    q, k, v, do = inputs.bwd_inputs(1, 2, 1, 0, 130, D, 3)
     q, k, v, do = (t.to(d) for t in (q, k, v, do))
     o = torch.empty_like(q)
     lse = torch.empty(1, 2, 0, device=d)
@@ -107,7 +111,7 @@ def test_empty_query_or_key_side():
     torch.cuda.synchronize()
     assert ea.read_device_status(0) == 0
     assert not dk.any() and not dv.any()          # no query: zero gradients for K and V
-    q, k, v, do = inputs.bwd_inputs(1, 2, 1, 70, 0, 64, 4)
+    q, k, v, do = inputs.bwd_inputs(1, 2, 1, 70, 0, D, 4)
     q, k, v, do = (t.to(d) for t in (q, k, v, do))
     o, lse = ea.fwd(q, k, v, causal=False)
     dq = torch.full_like(q, 7.0)

@@ -79,6 +79,15 @@ def test_growing_row_max_rescales(D):
                 o_max_abs=bf16_arith_bound(v.float().abs().max().item()))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_persistent_walk_with_keyless_tiles(D):
+    """More units than SMs (each CTA walks several), causal with Nq > Nk so
+    that the first units' tiles see no key at all (O = 0, LSE = -inf) while
+    later units of the same CTA do full work: the barrier counts that carry
+    across units (Q tile free, O read, last product) must stay in step."""
+    _check_full(4, 64, 8, 700, 300, D, True, seed=71 + D)
+
+
 def test_no_keys():
     dev = torch.device("cuda:0")
     q, k, v = inputs.prefill_inputs(1, 2, 2, 100, 0, 128, 128, seed=3)
