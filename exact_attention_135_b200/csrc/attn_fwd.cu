@@ -88,10 +88,15 @@ struct FwdCfg {
   static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
   static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
   static constexpr int ISSUE_REGS = 56;
+  // setmaxnreg.inc draws on the registers the block was launched with
+  // (THREADS x LAUNCH_REGS), not on the SM's 65,536: the split must fit
+  // that total, or the increase waits forever.
   static constexpr int SOFTMAX_REGS =
-      ((65536 - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8 > 248
+      ((THREADS * LAUNCH_REGS - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8 > 248
           ? 248
-          : ((65536 - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8;
+          : ((THREADS * LAUNCH_REGS - 128 * ISSUE_REGS) / (SOFTMAX_WARPS * 32)) / 8 * 8;
+  static_assert(NT == 1 || 128 * ISSUE_REGS + SOFTMAX_WARPS * 32 * SOFTMAX_REGS <= THREADS * LAUNCH_REGS,
+                "register split within the launch allocation");
   // TMEM columns: tile t owns [t*TILE_COLS, ...): NSL S buffers of BN
   // columns, then O (D columns).
   static constexpr int TILE_COLS = 256;
