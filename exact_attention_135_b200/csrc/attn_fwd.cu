@@ -366,54 +366,60 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     int sc[NT] = {};      // score tiles of tile t before this unit
     int qld[NT] = {};     // Q loads of tile t consumed
     int orc[NT] = {};     // epilogues of tile t before this unit (arrivals on its O-read barrier)
+    int pre[NT] = {};     // score tiles of this unit issued while the previous one ran
+    bool qpre[NT] = {};   // Q of tile t for this unit already waited for then
     bool ok = true;
-    for (int k = 0, u; ok && (u = unit_index(blockIdx.x, gridDim.x, k, a.n_units)) >= 0; ++k) {
+    auto last_tile_of = [&](const int* nb, int j) {
+      int lt = -1;
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+        if (j < nb[t]) lt = t;
+      return lt;
+    };
+    // S(t, j) of a unit whose K blocks start at ring count kb and whose tile-t
+    // score tiles start at running count sb: Q_t K_j^T into S buffer (sb + j) % NSL.
+    auto issue_s = [&](int t, int j, int kb, int sb, const int* nb) -> bool {
+      const int kj = kb + j, st = kj % KST;
+      if (!warp_wait(bar(C::B_KF + st), (kj / KST) & 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const int c = sb + j;
+      const uint32_t d_tmem = tmem + t * C::TILE_COLS + (c % NSL) * BN;
+      const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / C::K_MMA; ++ks) {
+        // advance the start-address field (16-byte units) to k-step ks (32 bytes of a row)
+        const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
+        const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
+        if constexpr (C::FP8) mma_ss_f8(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+        else mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
+      }
+      mma_commit(bar(C::B_SF + t * NSL + (c % NSL)), leader);
+      if (t == last_tile_of(nb, j)) mma_commit(bar(C::B_KE + st), leader);
+      // O staged apart: the Q tile is free once the unit's last score tile is done
+      if (C::SEP_OSTAGE && j == nb[t] - 1) mma_commit(bar(C::B_QE + t), leader);
+      __syncwarp();
+      return true;
+    };
+    for (int k = 0, u = unit_index(blockIdx.x, gridDim.x, 0, a.n_units); ok && u >= 0; ++k) {
       const Unit x = unit_of(a, u, C::CAUSAL);
       int nblk[NT];
       const int nmax = unit_blocks(x, nblk);
+      const int un = unit_index(blockIdx.x, gridDim.x, k + 1, a.n_units);
+      int nblk_n[NT] = {};
+      if (un >= 0) unit_blocks(unit_of(a, un, C::CAUSAL), nblk_n);
+      int pre_n[NT] = {};
+      bool qpre_n[NT] = {};
 #pragma unroll
       for (int t = 0; t < NT; ++t)
-        if (ok && nblk[t] > 0) {
+        if (ok && nblk[t] > 0 && !qpre[t]) {
           ok = warp_wait(bar(C::B_QF + t), qld[t] & 1, abort_flag, a.status);
           ++qld[t];
         }
-
-      auto last_tile = [&](int j) {
-        int lt = -1;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-          if (j < nblk[t]) lt = t;
-        return lt;
-      };
-      // S(t, j) = Q_t K_j^T into S buffer (sc[t] + j) % NSL of tile t.
-      auto issue_s = [&](int t, int j) -> bool {
-        const int kj = kc + j, st = kj % KST;
-        if (!warp_wait(bar(C::B_KF + st), (kj / KST) & 1, abort_flag, a.status)) return false;
-        tc_fence_after();
-        const int c = sc[t] + j;
-        const uint32_t d_tmem = tmem + t * C::TILE_COLS + (c % NSL) * BN;
-        const uint64_t qdesc = sdesc_sw128(base + C::OFF_Q + t * C::Q_BYTES, 16, 1024);
-        const uint64_t kdesc = sdesc_sw128(base + C::OFF_K + st * C::KV_BYTES, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < D / C::K_MMA; ++ks) {
-          // advance the start-address field (16-byte units) to k-step ks (32 bytes of a row)
-          const uint32_t dq = ((ks >> 2) * C::Q_CHUNK + (ks & 3) * 32) >> 4;
-          const uint32_t dk = ((ks >> 2) * C::KV_CHUNK + (ks & 3) * 32) >> 4;
-          if constexpr (C::FP8) mma_ss_f8(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
-          else mma_ss(d_tmem, qdesc + dq, kdesc + dk, idesc_s, ks > 0, leader);
-        }
-        mma_commit(bar(C::B_SF + t * NSL + (c % NSL)), leader);
-        if (t == last_tile(j)) mma_commit(bar(C::B_KE + st), leader);
-        // O staged apart: the Q tile is free once the unit's last score tile is done
-        if (C::SEP_OSTAGE && j == nblk[t] - 1) mma_commit(bar(C::B_QE + t), leader);
-        __syncwarp();
-        return true;
-      };
-
       for (int i = 0; ok && i < NSL; ++i)
 #pragma unroll
         for (int t = 0; t < NT; ++t)
-          if (ok && i < nblk[t]) ok = issue_s(t, i);
+          if (ok && i < nblk[t] && i >= pre[t]) ok = issue_s(t, i, kc, sc[t], nblk);
 
       for (int j = 0; ok && j < nmax; ++j) {
         const int vj = vc + j, st = vj % VST;
@@ -445,9 +451,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mma_commit(bar(C::B_OD + t), leader);
           if (j == nblk[t] - 1) mma_commit(bar(C::B_OF + t), leader);
-          if (t == last_tile(j)) mma_commit(bar(C::B_VE + st), leader);
+          if (t == last_tile_of(nblk, j)) mma_commit(bar(C::B_VE + st), leader);
           __syncwarp();
-          if (j + NSL < nblk[t]) ok = issue_s(t, j + NSL);
+          if (j + NSL < nblk[t]) {
+            ok = issue_s(t, j + NSL, kc, sc[t], nblk);
+          } else if (C::SEP_OSTAGE && j == nblk[t] - 1 && un >= 0 && nblk_n[t] > 0) {
+            // Tile t is done with this unit.  Its score tiles of the next unit
+            // are issued now if that unit's Q and K blocks have landed (tested,
+            // not waited for), so they are computed during this tile's
+            // epilogue instead of after the other tile's last products.  The
+            // S buffers they overwrite held this unit's last blocks, whose
+            // P V products were issued above.  (With O staged in the Q tile,
+            // the next Q cannot have landed before this tile's epilogue.)
+            if (__all_sync(0xffffffffu, mbar_try_wait(bar(C::B_QF + t), qld[t] & 1))) {
+              ++qld[t];
+              qpre_n[t] = true;
+              tc_fence_after();
+              for (int i = 0; ok && i < NSL && i < nblk_n[t]; ++i) {
+                const int kj = kc + nmax + i;
+                if (!__all_sync(0xffffffffu, mbar_try_wait(bar(C::B_KF + kj % KST), (kj / KST) & 1))) break;
+                ok = issue_s(t, i, kc + nmax, sc[t] + nblk[t], nblk_n);
+                ++pre_n[t];
+              }
+            }
+          }
         }
       }
       kc += nmax;
@@ -456,7 +483,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int t = 0; t < NT; ++t) {
         sc[t] += nblk[t];
         orc[t] += tile_active(x, t) ? 1 : 0;
+        pre[t] = pre_n[t];
+        qpre[t] = qpre_n[t];
       }
+      u = un;
     }
     // Drain: no MMA may still run when TMEM is released.
     mma_commit(bar(C::B_DR), leader);
@@ -556,6 +586,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
       }
       if (n > 0) ++ofc;
+      // O staged apart: the previous unit's TMA store of this staging area
+      // is waited for here, just before it is rewritten, not right after it
+      // was issued.
+      if (C::SEP_OSTAGE && wq == 0 && lane == 0) tma_store_wait_read();
       // The four warps of the tile take the same path from here on (a warp
       // whose wait failed must not leave the others at a named barrier); the
       // barrier also orders this staging after the previous unit's TMA store
@@ -598,7 +632,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int ch = 0; ch < D / 64; ++ch) tma_store_4d(&tm_o, stage + ch * C::Q_CHUNK, ch * 64, x.hq, r0, x.b);   // bf16 O
           tma_store_commit();
-          tma_store_wait_read();
+          if (!C::SEP_OSTAGE) tma_store_wait_read();
         }
         if (!C::SEP_OSTAGE) mbar_arrive(bar(C::B_QE + t));   // the Q tile may be reloaded
       }
@@ -607,6 +641,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             (l_run > 0.f) ? (m_run - C::P_SHIFT + log2f(l_run)) * kLn2 : -INFINITY;
       __syncwarp();
     }
+    // the last TMA store of O has read its staging before the CTA ends
+    if (C::SEP_OSTAGE && wq == 0 && lane == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
