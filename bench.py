@@ -61,12 +61,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu capture of the same launch; see profiles/.  Set to None whenever the
 # kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "prefill": None,                    # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload: to capture
-    "prefill_c4": None,                 # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload: to capture
+    "prefill": 369158912 + 106672896,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
+    "prefill_c4": 151093504 + 101837824,   # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload
     "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
-    "bwd": 2360328704 + 1253101056,     # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
-    "fp8": None,                        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3: to capture
+    "bwd": None,                        # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward): to capture
+    "fp8": 100876800 + 89678080,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
 }
 # Timed regions longer than this run under the power cap: compare with the
 # sustained peak rather than the burst one.

@@ -49,6 +49,7 @@
 
 #include "host_common.h"
 #include "sm100.cuh"
+#include "softmax_row.cuh"
 
 namespace ea {
 namespace bwd {
@@ -827,14 +828,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t s[64];
       tmem_ld64_sync(tS, s);
       uint32_t pk[32];
+      // Pairs of columns: 5 of every 16 take 2^x on the FMA pipe (the
+      // polynomial of sm100.cuh), the rest on the MUFU unit, whose throughput
+      // otherwise sets this pass.  A column whose row saw no key (LSE2 = +inf)
+      // gives exactly 0 either way.
+      const uint64_t k2 = f2_pack(sl2, sl2);
+      auto exp2_pair = [&](int c, uint64_t x, uint32_t la, uint32_t lb, float& pa, float& pb) {
+        if (poly_pair(c)) {
+          exp2_poly_x2(x, pa, pb);
+          if (__uint_as_float(la) == INFINITY) pa = 0.f;
+          if (__uint_as_float(lb) == INFINITY) pb = 0.f;
+        } else {
+          float xa, xb;
+          f2_unpack(x, xa, xb);
+          pa = ex2(xa);
+          pb = ex2(xb);
+        }
+      };
 #pragma unroll
       for (int j = 0; j < 64; j += 4) {
         uint32_t l0, l1, l2, l3;
         ld_shared_v4(rows_s + j * 4, l0, l1, l2, l3);
-        const float p0 = ex2(fmaf(__uint_as_float(s[j + 0]), sl2, -__uint_as_float(l0)));
-        const float p1 = ex2(fmaf(__uint_as_float(s[j + 1]), sl2, -__uint_as_float(l1)));
-        const float p2 = ex2(fmaf(__uint_as_float(s[j + 2]), sl2, -__uint_as_float(l2)));
-        const float p3 = ex2(fmaf(__uint_as_float(s[j + 3]), sl2, -__uint_as_float(l3)));
+        const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(s[j + 0]), __uint_as_float(s[j + 1])), k2,
+                                    f2_pack(-__uint_as_float(l0), -__uint_as_float(l1)));
+        const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(s[j + 2]), __uint_as_float(s[j + 3])), k2,
+                                    f2_pack(-__uint_as_float(l2), -__uint_as_float(l3)));
+        float p0, p1, p2, p3;
+        exp2_pair(j / 2, x01, l0, l1, p0, p1);
+        exp2_pair(j / 2 + 1, x23, l2, l3, p2, p3);
         pk[j / 2] = pack_bf16x2(p0, p1);
         pk[j / 2 + 1] = pack_bf16x2(p2, p3);
       }

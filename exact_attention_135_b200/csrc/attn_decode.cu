@@ -721,12 +721,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// One CTA per (sequence, group of 16 heads): merges the partial results of a
+// One CTA per (sequence, group of 4 heads): merges the partial results of a
 // sequence that several CTA pairs shared; writes O = 0, LSE = -inf for an
 // empty sequence; leaves sequences written by the split kernel untouched.
-constexpr int COMBINE_HEADS = 16;
+// A long sequence in a small batch is spread over up to all CTA pairs, so
+// every step is parallel over the pieces: the piece list is built by one
+// thread per pair, the weights by one thread per (head, piece) and one warp
+// per head, and the weighted sum issues the loads of several pieces at once.
+constexpr int COMBINE_HEADS = 4;
 constexpr int COMBINE_THREADS = 256;
 constexpr int MAX_PARTS = 128;   // >= CTA pairs, so a sequence never has more pieces
+constexpr int COMBINE_UNROLL = 4;   // pieces whose loads are in flight together
+static_assert(MAX_PARTS <= COMBINE_THREADS && COMBINE_HEADS <= COMBINE_THREADS / 32, "combine thread map");
 
 __global__ void __launch_bounds__(COMBINE_THREADS)
     decode_combine_kernel(const Args a) {
@@ -735,7 +741,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int h0 = blockIdx.y * COMBINE_HEADS;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = a.ws_pref[a.B];
   const int s0 = a.ws_pref[b], s1 = a.ws_pref[b + 1];
   if (s1 == s0) {
@@ -748,65 +754,95 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
   if (p_lo == p_hi) return;
   __shared__ float w_s[COMBINE_HEADS][MAX_PARTS];
   __shared__ int slot_s[MAX_PARTS];
-  __shared__ int nparts_s;
-  if (tid == 0) {
-    // pairs with an empty range (fewer pages than pairs) hold no piece
-    int n = 0;
-    for (int p = p_lo; p <= p_hi && n < MAX_PARTS; ++p) {
-      const int r0 = range_start(p, T, a.pairs);
-      if (range_start(p + 1, T, a.pairs) == r0) continue;
-      slot_s[n++] = 2 * p + ((p == p_lo && s0 != r0) ? 1 : 0);
-    }
-    nparts_s = n;
+  __shared__ int wcount_s[COMBINE_THREADS / 32];
+  // Pieces in pair order; pairs with an empty range (fewer pages than
+  // pairs) hold none.  Thread i looks at pair p_lo + i.
+  const int npairs = min(p_hi - p_lo + 1, MAX_PARTS);
+  bool has = false;
+  int slot = 0;
+  if (tid < npairs) {
+    const int p = p_lo + tid;
+    const int r0 = range_start(p, T, a.pairs);
+    has = range_start(p + 1, T, a.pairs) > r0;
+    slot = 2 * p + ((p == p_lo && s0 != r0) ? 1 : 0);
+  }
+  const uint32_t ballot = __ballot_sync(0xffffffffu, has);
+  if (lane == 0) wcount_s[warp] = __popc(ballot);
+  __syncthreads();
+  int before = 0, nparts = 0;
+#pragma unroll
+  for (int w = 0; w < COMBINE_THREADS / 32; ++w) {
+    before += (w < warp) ? wcount_s[w] : 0;
+    nparts += wcount_s[w];
+  }
+  if (has) slot_s[before + __popc(ballot & ((1u << lane) - 1u))] = slot;
+  __syncthreads();
+  // LSE of every (head, piece), then one warp per head: max, weights, LSE
+  for (int i = tid; i < COMBINE_HEADS * nparts; i += COMBINE_THREADS) {
+    const int hh = i / nparts, j = i - hh * nparts;
+    w_s[hh][j] = a.ws_lse[(size_t)slot_s[j] * HQ + h0 + hh];
   }
   __syncthreads();
-  const int nparts = nparts_s;
-  if (tid < COMBINE_HEADS) {
-    const int h = h0 + tid;
+  if (warp < COMBINE_HEADS) {
     float mx = -INFINITY;
-    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) mx = fmaxf(mx, a.ws_lse[(size_t)slot_s[i] * HQ + h]);
+    for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, w_s[warp][j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float sum = 0.f;
-    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) {
-      const float e = (mx == -INFINITY) ? 0.f : expf(a.ws_lse[(size_t)slot_s[i] * HQ + h] - mx);
-      w_s[tid][i] = e;
+    for (int j = lane; j < nparts; j += 32) {
+      const float e = (mx == -INFINITY) ? 0.f : expf(w_s[warp][j] - mx);
+      w_s[warp][j] = e;
       sum += e;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    for (int i = 0; i < nparts && i < MAX_PARTS; ++i) w_s[tid][i] *= inv;
-    a.lse[(size_t)b * HQ + h] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    for (int j = lane; j < nparts; j += 32) w_s[warp][j] *= inv;
+    if (lane == 0) a.lse[(size_t)b * HQ + h0 + warp] = sum > 0.f ? mx + logf(sum) : -INFINITY;
   }
   __syncthreads();
-  // 16 heads x 512 columns: each thread owns OUT_PER_THREAD groups of 4
-  // columns (head hh = tid / 128 + 2k, columns 4 (tid % 128) ..), and the
-  // loads of one piece for all of them are issued together, so a piece costs
-  // one memory latency rather than one per group.
+  // COMBINE_HEADS x 512 columns as float4 groups: thread tid owns groups
+  // tid + COMBINE_THREADS k (head g / 128, columns 4 (g % 128) ..).
   constexpr int OUT_PER_THREAD = COMBINE_HEADS * DV / 4 / COMBINE_THREADS;
-  static_assert(OUT_PER_THREAD * COMBINE_THREADS * 4 == COMBINE_HEADS * DV && COMBINE_THREADS % (DV / 4) == 0,
-                "combine thread map");
-  const int c4 = tid % (DV / 4), hh0 = tid / (DV / 4);
-  constexpr int HH_STEP = COMBINE_THREADS / (DV / 4);
+  static_assert(OUT_PER_THREAD * COMBINE_THREADS * 4 == COMBINE_HEADS * DV, "combine output map");
   float4 acc[OUT_PER_THREAD];
+  const float* src0[OUT_PER_THREAD];
+  int hh_of[OUT_PER_THREAD];
 #pragma unroll
-  for (int k = 0; k < OUT_PER_THREAD; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < nparts && j < MAX_PARTS; ++j) {
-    const float* src = a.ws_o + ((size_t)slot_s[j] * HQ + h0) * DV + c4 * 4;
-    float4 v[OUT_PER_THREAD];
+  for (int k = 0; k < OUT_PER_THREAD; ++k) {
+    const int g = tid + COMBINE_THREADS * k;
+    hh_of[k] = g / (DV / 4);
+    src0[k] = a.ws_o + ((size_t)h0 + hh_of[k]) * DV + (g % (DV / 4)) * 4;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int j0 = 0; j0 < nparts; j0 += COMBINE_UNROLL) {
+    float4 v[COMBINE_UNROLL][OUT_PER_THREAD];
 #pragma unroll
-    for (int k = 0; k < OUT_PER_THREAD; ++k)
-      v[k] = *reinterpret_cast<const float4*>(src + (size_t)(hh0 + HH_STEP * k) * DV);
+    for (int u = 0; u < COMBINE_UNROLL; ++u) {
+      const int j = j0 + u;
+      const size_t off = (size_t)slot_s[j < nparts ? j : j0] * HQ * DV;
 #pragma unroll
-    for (int k = 0; k < OUT_PER_THREAD; ++k) {
-      const float wgt = w_s[hh0 + HH_STEP * k][j];
-      acc[k].x += wgt * v[k].x;
-      acc[k].y += wgt * v[k].y;
-      acc[k].z += wgt * v[k].z;
-      acc[k].w += wgt * v[k].w;
+      for (int k = 0; k < OUT_PER_THREAD; ++k)
+        v[u][k] = j < nparts ? *reinterpret_cast<const float4*>(src0[k] + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < COMBINE_UNROLL; ++u) {
+      const int j = j0 + u;
+      if (j >= nparts) break;
+#pragma unroll
+      for (int k = 0; k < OUT_PER_THREAD; ++k) {
+        const float wgt = w_s[hh_of[k]][j];
+        acc[k].x += wgt * v[u][k].x;
+        acc[k].y += wgt * v[u][k].y;
+        acc[k].z += wgt * v[u][k].z;
+        acc[k].w += wgt * v[u][k].w;
+      }
     }
   }
 #pragma unroll
   for (int k = 0; k < OUT_PER_THREAD; ++k) {
-    __nv_bfloat162* dst =
-        reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh0 + HH_STEP * k) * DV + c4 * 4);
+    const int g = tid + COMBINE_THREADS * k;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh_of[k]) * DV + (g % (DV / 4)) * 4);
     dst[0] = __floats2bfloat162_rn(acc[k].x, acc[k].y);
     dst[1] = __floats2bfloat162_rn(acc[k].z, acc[k].w);
   }
@@ -827,7 +863,9 @@ inline WsLayout ws_layout(int B, int pairs) {
   return w;
 }
 
-inline int pairs_for_sms(int sms) { return sms >= 2 ? sms / 2 : 0; }
+// CTA pairs of the split plan: one per two SMs, at most MAX_PARTS (the
+// combine merges up to MAX_PARTS pieces of a sequence).
+inline int pairs_for_sms(int sms) { return sms >= 2 ? (sms / 2 < MAX_PARTS ? sms / 2 : MAX_PARTS) : 0; }
 
 }  // namespace dec
 }  // namespace ea

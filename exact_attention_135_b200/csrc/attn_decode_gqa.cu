@@ -505,9 +505,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // One CTA per (sequence, KV head): merges the partial results of a unit that
 // several workers shared, writes O = 0 and LSE = -inf for an empty sequence,
 // leaves units written by the decode kernel untouched.  The number of pieces
-// is not bounded: they are taken in chunks of COMBINE_CHUNK, and each chunk's
-// slots and weights are computed once into shared memory, so the loop over
-// output elements only reads them.
+// is not bounded: workers are taken in chunks of COMBINE_CHUNK, and each
+// chunk's pieces, slots and weights are compacted into shared memory once, so
+// the loop over output elements only reads them.
 constexpr int COMBINE_THREADS = 128;
 constexpr int COMBINE_CHUNK = 128;
 constexpr int COMBINE_OUT = 8;   // output elements per thread: G * D <= 8 * 128
@@ -540,6 +540,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS) gqa_combine_kernel(const Args
   __shared__ float s_red[COMBINE_THREADS / 32][8];
   __shared__ float s_max[8], s_inv[8];
   __shared__ int s_slot[COMBINE_CHUNK];
+  __shared__ int s_cnt[COMBINE_THREADS / 32];
   __shared__ float s_w[8][COMBINE_CHUNK];
 
   // per-head maximum, then sum of exp(lse - max), over all pieces (in parallel over pieces)
@@ -582,35 +583,56 @@ __global__ void __launch_bounds__(COMBINE_THREADS) gqa_combine_kernel(const Args
     __syncthreads();
   }
 
-  // O = sum over pieces of weight * partial O, one chunk of pieces at a time
+  // O = sum over pieces of weight * partial O, one chunk of workers at a
+  // time: the chunk's pieces are first compacted (most workers of a short
+  // sequence in a small batch hold none), then the loads of two pieces for
+  // all of a thread's outputs are issued together.
   float out[COMBINE_OUT];
 #pragma unroll
   for (int k = 0; k < COMBINE_OUT; ++k) out[k] = 0.f;
   for (int c0 = 0; c0 < n; c0 += COMBINE_CHUNK) {
     const int cn = min(COMBINE_CHUNK, n - c0);
-    if (tid < cn) {
-      const int sl = slot_of(w_lo + c0 + tid);
-      s_slot[tid] = sl;
+    const int sl = tid < cn ? slot_of(w_lo + c0 + tid) : -1;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, sl >= 0);
+    if (lane == 0) s_cnt[warp] = __popc(ballot);
+    __syncthreads();
+    int before = 0, m = 0;
+#pragma unroll
+    for (int w = 0; w < COMBINE_THREADS / 32; ++w) {
+      before += (w < warp) ? s_cnt[w] : 0;
+      m += s_cnt[w];
+    }
+    if (sl >= 0) {
+      const int pos = before + __popc(ballot & ((1u << lane) - 1u));
+      s_slot[pos] = sl;
 #pragma unroll
       for (int h = 0; h < 8; ++h) {
         if (h >= G) break;
-        s_w[h][tid] = (sl < 0 || s_max[h] == -INFINITY)
-                          ? 0.f
-                          : expf(a.ws_lse[(size_t)sl * G + h] - s_max[h]) * s_inv[h];
+        s_w[h][pos] = s_max[h] == -INFINITY ? 0.f : expf(a.ws_lse[(size_t)sl * G + h] - s_max[h]) * s_inv[h];
       }
     }
     __syncthreads();
+    for (int j0 = 0; j0 < m; j0 += 2) {
+      const bool two = j0 + 1 < m;
+      const int j1 = two ? j0 + 1 : j0;   // v1 is 0 when there is no second piece
+      const float* src0 = a.ws_o + (size_t)s_slot[j0] * G * D;
+      const float* src1 = a.ws_o + (size_t)s_slot[j1] * G * D;
+      float v0[COMBINE_OUT], v1[COMBINE_OUT];
 #pragma unroll
-    for (int k = 0; k < COMBINE_OUT; ++k) {
-      const int i = tid + k * COMBINE_THREADS;
-      if (i >= G * D) break;
-      const int h = i / D;
-      float acc = out[k];
-      for (int j = 0; j < cn; ++j) {
-        const int sl = s_slot[j];
-        if (sl >= 0) acc += s_w[h][j] * a.ws_o[(size_t)sl * G * D + i];
+      for (int k = 0; k < COMBINE_OUT; ++k) {
+        const int i = tid + k * COMBINE_THREADS;
+        const bool in = i < G * D;
+        v0[k] = in ? src0[i] : 0.f;
+        v1[k] = (in && two) ? src1[i] : 0.f;
       }
-      out[k] = acc;
+#pragma unroll
+      for (int k = 0; k < COMBINE_OUT; ++k) {
+        const int i = tid + k * COMBINE_THREADS;
+        if (i < G * D) {
+          const int h = i / D;
+          out[k] += s_w[h][j0] * v0[k] + s_w[h][j1] * v1[k];
+        }
+      }
     }
     __syncthreads();
   }
