@@ -77,6 +77,10 @@ struct FwdCfg {
   // (0, 2^(THR + SHIFT)] = (0, 256]: inside e4m3's range (max 448) and mostly
   // above its smallest normal (2^-6).
   static constexpr float RESCALE_THR = FP8 ? 4.0f : 8.0f;
+  // Column pairs c with (c mod 16) >= POLY_T take exp2 on the FMA pipe in
+  // full blocks: 6 of 16 for bf16 at head dim 128, 5 of 16 otherwise (a sweep
+  // of 3..7 of 16: head dim 128 bf16 +2 % at 6, head dim 64 and FP8 best at 5).
+  static constexpr int POLY_T = (D == 128 && !FP8) ? 10 : 11;
   static constexpr float P_SHIFT = FP8 ? 4.0f : 0.0f;
   static constexpr int SOFTMAX_WARPS = 4 * NT;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;       // K loads
@@ -546,9 +550,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // and must give exactly 0); full blocks send part of the work to the FMA pipe.
         float sum;
         if constexpr (C::FP8)
-          sum = need_mask ? exp_row_e4m3<BN, false>(s, p, sl2, m_eff) : exp_row_e4m3<BN, true>(s, p, sl2, m_eff);
+          sum = need_mask ? exp_row_e4m3<BN, false>(s, p, sl2, m_eff)
+                          : exp_row_e4m3<BN, true, C::POLY_T>(s, p, sl2, m_eff);
         else
-          sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true>(s, p, sl2, m_eff);
+          sum = need_mask ? exp_row<BN, false>(s, p, sl2, m_eff) : exp_row<BN, true, C::POLY_T>(s, p, sl2, m_eff);
         l_run = l_run * alpha + sum;
         m_run = m_use;
         static_assert(C::P_WORDS % 32 == 0, "P rows are stored 32 columns at a time");

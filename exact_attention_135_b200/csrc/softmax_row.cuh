@@ -24,13 +24,13 @@ __device__ __forceinline__ float row_max(const uint32_t* s) {
   return fmaxf(max3f(m0, m1, m2), m3);
 }
 
-// Pairs of columns whose exp2 runs on the FMA pipe in full blocks: 5 of every
-// 16 pairs, which balances the MUFU unit against the issue slots the
-// polynomial costs.
-__device__ __forceinline__ constexpr bool poly_pair(int c) { return (c & 15) >= 11; }
+// Pairs of columns whose exp2 runs on the FMA pipe in full blocks: pairs
+// with (c mod 16) >= T, 5 of every 16 by default, which balances the MUFU
+// unit against the issue slots the polynomial costs.
+__device__ __forceinline__ constexpr bool poly_pair(int c, int T = 11) { return (c & 15) >= T; }
 
 // p = 2^(s * sl2 - m) for one row, packed to bf16 pairs; returns the fp32 sum.
-template <int N, bool MIXED>
+template <int N, bool MIXED, int POLY_T = 11>
 __device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float sl2, float m) {
   const uint64_t k2 = f2_pack(sl2, sl2);
   const uint64_t nm2 = f2_pack(-m, -m);
@@ -39,7 +39,7 @@ __device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float s
   for (int c = 0; c < N / 2; ++c) {
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), k2, nm2);
     float p0, p1;
-    if (MIXED && poly_pair(c)) {
+    if (MIXED && poly_pair(c, POLY_T)) {
       exp2_poly_x2(x, p0, p1);
     } else {
       float x0, x1;
@@ -59,7 +59,7 @@ __device__ __forceinline__ float exp_row(const uint32_t* s, uint32_t* p, float s
 
 // The same with p packed four to a word as e4m3 bytes (column 4w + i in
 // byte i of word w), the layout of an 8-bit A operand in tensor memory.
-template <int N, bool MIXED>
+template <int N, bool MIXED, int POLY_T = 11>
 __device__ __forceinline__ float exp_row_e4m3(const uint32_t* s, uint32_t* p, float sl2, float m) {
   const uint64_t k2 = f2_pack(sl2, sl2);
   const uint64_t nm2 = f2_pack(-m, -m);
@@ -68,7 +68,7 @@ __device__ __forceinline__ float exp_row_e4m3(const uint32_t* s, uint32_t* p, fl
   for (int c = 0; c < N / 2; ++c) {
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), k2, nm2);
     float p0, p1;
-    if (MIXED && poly_pair(c)) {
+    if (MIXED && poly_pair(c, POLY_T)) {
       exp2_poly_x2(x, p0, p1);
     } else {
       float x0, x1;
