@@ -61,11 +61,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu capture of the same launch; see profiles/.  Set to None whenever the
 # kernel changes until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "prefill": 369158912 + 106672896,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
+    "prefill": 364641536 + 105544448,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
     "prefill_c4": 151093504 + 101837824,   # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload
     "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
-    "bwd": None,                        # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward): to capture
+    "bwd": 2336795392 + 1236150272,     # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
     "fp8": 100876800 + 89678080,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
 }
 # Timed regions longer than this run under the power cap: compare with the

@@ -721,19 +721,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// One CTA per (sequence, group of 4 heads): merges the partial results of a
+// One CTA per (sequence, group of 8 heads): merges the partial results of a
 // sequence that several CTA pairs shared; writes O = 0, LSE = -inf for an
 // empty sequence; leaves sequences written by the split kernel untouched.
 // A long sequence in a small batch is spread over up to all CTA pairs, so
 // every step is parallel over the pieces: the piece list is built by one
 // thread per pair, the weights by one thread per (head, piece) and one warp
 // per head, and the weighted sum issues the loads of several pieces at once.
-constexpr int COMBINE_HEADS = 4;
+// Two shapes (heads per CTA x pieces in flight): 8 x 2 when the batch gives
+// at least two CTAs per SM, 4 x 4 for smaller batches, whose few sequences
+// are spread over many pairs (a sweep of 4, 8 and 16 heads with 2 or 4
+// pieces: 139.6-141.8 us for the whole decode of a 64-sequence batch, the
+// lowest at 8 x 2; 40-55 us for four sequences of 70, 0, 200 and 6000
+// tokens, the combine alone 20 us at 4 x 4 and 35 us at 8 x 2 under ncu).
 constexpr int COMBINE_THREADS = 256;
 constexpr int MAX_PARTS = 128;   // >= CTA pairs, so a sequence never has more pieces
-constexpr int COMBINE_UNROLL = 4;   // pieces whose loads are in flight together
-static_assert(MAX_PARTS <= COMBINE_THREADS && COMBINE_HEADS <= COMBINE_THREADS / 32, "combine thread map");
+static_assert(MAX_PARTS <= COMBINE_THREADS, "combine thread map");
 
+template <int COMBINE_HEADS, int COMBINE_UNROLL>
 __global__ void __launch_bounds__(COMBINE_THREADS)
     decode_combine_kernel(const Args a) {
   // Launched as a programmatic dependent of the split kernel: wait here until
@@ -783,22 +788,22 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
     w_s[hh][j] = a.ws_lse[(size_t)slot_s[j] * HQ + h0 + hh];
   }
   __syncthreads();
-  if (warp < COMBINE_HEADS) {
+  for (int hh = warp; hh < COMBINE_HEADS; hh += COMBINE_THREADS / 32) {
     float mx = -INFINITY;
-    for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, w_s[warp][j]);
+    for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, w_s[hh][j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float sum = 0.f;
     for (int j = lane; j < nparts; j += 32) {
-      const float e = (mx == -INFINITY) ? 0.f : expf(w_s[warp][j] - mx);
-      w_s[warp][j] = e;
+      const float e = (mx == -INFINITY) ? 0.f : expf(w_s[hh][j] - mx);
+      w_s[hh][j] = e;
       sum += e;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    for (int j = lane; j < nparts; j += 32) w_s[warp][j] *= inv;
-    if (lane == 0) a.lse[(size_t)b * HQ + h0 + warp] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    for (int j = lane; j < nparts; j += 32) w_s[hh][j] *= inv;
+    if (lane == 0) a.lse[(size_t)b * HQ + h0 + hh] = sum > 0.f ? mx + logf(sum) : -INFINITY;
   }
   __syncthreads();
   // COMBINE_HEADS x 512 columns as float4 groups: thread tid owns groups
@@ -949,8 +954,10 @@ extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const 
   // The combine is a programmatic dependent launch: its CTAs are scheduled as
   // the split kernel's CTAs retire and wait (griddepcontrol.wait) for that
   // grid's completion, instead of the stream's full launch gap.
+  // a batch too small to give two 8-head CTAs per SM takes 4 heads per CTA
+  const bool small_batch = (long long)units * (HQ / 8) < 4LL * pairs;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(units, HQ / COMBINE_HEADS);
+  cfg.gridDim = dim3(units, HQ / (small_batch ? 4 : 8));
   cfg.blockDim = dim3(COMBINE_THREADS);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -959,7 +966,9 @@ extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, a) != cudaSuccess) return ATTN_ERR_CUDA;
+  const cudaError_t e = small_batch ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<4, 4>, a)
+                                    : cudaLaunchKernelEx(&cfg, decode_combine_kernel<8, 2>, a);
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

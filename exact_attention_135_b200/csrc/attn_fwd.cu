@@ -10,9 +10,12 @@
 // first score tile overlap the previous unit's epilogue.  Per unit it streams the
 // KV head's K/V in blocks of BN keys through shared memory:
 //
-//   producer warp   TMA: Q tiles once, then a ring of K and V blocks
+//   producer warps  TMA: a ring of K blocks, a ring of V blocks, and each
+//                   unit's Q tiles once their buffers are free again
 //   MMA warp        one thread issues tcgen05.mma:  S = Q K^T  into TMEM,
-//                   then O += P V with P read from TMEM (it overwrites S)
+//                   then O += P V with P read from TMEM (it overwrites S);
+//                   with O staged apart, a tile's first score tiles of the
+//                   next unit follow its last P V of the current unit
 //   softmax WGs     one warpgroup per Q tile, one TMEM lane (= query row) per
 //                   thread: load S, mask, running max, p = 2^(s*scale*log2e - m),
 //                   running sum, P -> bf16 -> TMEM; rescale O only when the
