@@ -63,7 +63,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_BYTES = {
     "prefill": 364641536 + 105544448,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
     "prefill_c4": 151093504 + 101837824,   # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload
+    "prefill_c2": 37816320 + 63232,     # attn_fwd_kernel<D=64, causal> (persistent), GPT-2-small shape
     "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
+    "mtp": 581064192 + 28656128,        # decode_split_kernel, MLA decode workload with 2 query tokens per sequence
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
     "bwd": 2336795392 + 1236150272,     # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
     "fp8": 100876800 + 89678080,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
@@ -470,7 +472,8 @@ def run_gpu(args):
                                         NCU_TRAFFIC_BYTES.get("prefill_c4"))
     if "prefill_c2" in by:
         objs["prefill_c2"] = tensor_obj(by["prefill_c2"], "attention TFLOP/s (prefill, GPT-2-small shape)",
-                                        "attn_fwd_kernel<D=64,causal>", bf16_peak, bf16_kind)
+                                        "attn_fwd_kernel<D=64,causal>", bf16_peak, bf16_kind,
+                                        NCU_TRAFFIC_BYTES.get("prefill_c2"))
     if "prefill_c1" in by:
         p = by["prefill_c1"]
         o = tensor_obj(p, "attention TFLOP/s (prefill, tiny)", "attn_fwd_kernel<D=64,non-causal>", bf16_peak,
