@@ -67,7 +67,7 @@ NCU_TRAFFIC_BYTES = {
     "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
     "mtp": 581064192 + 28656128,        # decode_split_kernel, MLA decode workload with 2 query tokens per sequence
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
-    "bwd": 2336795392 + 1236150272,     # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
+    "bwd": 665277184 + 338907392,       # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
     "fp8": 100876800 + 89678080,        # attn_fwd_kernel<D=128, causal, fp8>, same shape in E4M3
 }
 # Timed regions longer than this run under the power cap: compare with the

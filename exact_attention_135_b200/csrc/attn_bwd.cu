@@ -20,7 +20,8 @@
 //   attn_bwd_kernel (D = 64, below)
 //   bwd_dqt_kernel / bwd_dq_kernel   dQ accumulator -> bf16
 //
-// Both attention kernels run one CTA per (key block of 128, KV head, batch).
+// Both attention kernels run one CTA per (key block of 128, KV head, batch),
+// in the order that unit_pos and choose_head_group describe.
 // dK and dV stay in TMEM while the CTA walks every query block of every query
 // head of the group that sees its keys; each step's dQ contribution is added
 // to the accumulator by a TMA reduce-add (at L2, coalesced whole tiles).
@@ -46,6 +47,12 @@
 // so the next step's S^T is computed while WG0 still forms dS_i, and dQ's
 // drain overlaps the next step's softmax work.
 #include <math.h>
+
+#include <algorithm>
+#include <functional>
+#include <mutex>
+#include <queue>
+#include <vector>
 
 #include "host_common.h"
 #include "sm100.cuh"
@@ -111,8 +118,30 @@ struct Args {
   __nv_bfloat16* dv;     // [B, Nk, Hkv, D]
   int* status;
   int B, Hq, Hkv, Nq, Nk, group, n_qblk, n_kblk, causal_off;
+  int head_group;        // heads (batch, KV head pairs) per group of the unit order
   float scale, scale_log2;
 };
+
+// Work unit u -> (key block, KV head, batch).  A head is one (batch, KV head)
+// pair p = b * Hkv + hk.  Heads are taken head_group at a time, and inside a
+// group the key block is the slower index, so with a causal mask the key
+// blocks that see the most query blocks start first.  A group smaller than
+// all heads makes the CTAs resident at once share the Q, dO and dQ
+// accumulator rows of fewer heads, which then stay in L2 from one CTA to the
+// next; head_group = Hkv * B is key block slowest over every head.
+struct UnitPos {
+  int kb, hk, b;
+};
+__device__ __forceinline__ UnitPos unit_pos(int u, const Args& a) {
+  const int g = a.head_group;
+  const int per_group = g * a.n_kblk;
+  const int grp = u / per_group;
+  const int r = u - grp * per_group;
+  const int p0 = grp * g;
+  const int gs = min(g, a.Hkv * a.B - p0);   // the last group may be smaller
+  const int p = p0 + r % gs;
+  return {r / gs, p % a.Hkv, p / a.Hkv};
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -139,12 +168,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   auto do_off = [&](int st) -> uint32_t { return base + C::OFF_STAGE + (2 * st + 1) * TILE; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Unit order: key block slowest, so with a causal mask the blocks that see
-  // the most query blocks (the first ones) start first.
-  const int u = blockIdx.x;
-  const int kb = u / (a.Hkv * a.B);
-  const int hk = (u % (a.Hkv * a.B)) % a.Hkv;
-  const int b = (u % (a.Hkv * a.B)) / a.Hkv;
+  const UnitPos up = unit_pos(blockIdx.x, a);
+  const int kb = up.kb, hk = up.hk, b = up.b;
   const int k0 = kb * C::BN;
   int qb_start = 0;
   if (C::CAUSAL) qb_start = max(0, (k0 - a.causal_off) / C::BM);   // first query block with a visible key
@@ -616,10 +641,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   auto rows_off = [&](int st) -> uint32_t { return base + C::OFF_ROWS + st * 512; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x;
-  const int kb = u / (a.Hkv * a.B);
-  const int hk = (u % (a.Hkv * a.B)) % a.Hkv;
-  const int b = (u % (a.Hkv * a.B)) / a.Hkv;
+  const UnitPos up = unit_pos(blockIdx.x, a);
+  const int kb = up.kb, hk = up.hk, b = up.b;
   const int k0 = kb * C::BN;
   int qb_start = 0;
   if (C::CAUSAL) qb_start = max(0, (k0 - a.causal_off) / BM);   // first query block with a visible key
@@ -1104,6 +1127,73 @@ __global__ void __launch_bounds__(256) bwd_dqt_kernel(const float* __restrict__ 
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// ---------------------------------------------------------------- unit order
+//
+// The grid has one CTA per unit and one CTA fits an SM, so the block
+// scheduler hands the units out in index order, each to the SM that frees
+// first.  Key block slowest over all heads puts the heaviest causal units
+// first (the best balance), but then the resident CTAs cover every head and
+// each later wave streams the Q, dO and dQ accumulator rows of every head
+// from DRAM again.  Grouping ceil(SMs / key blocks) heads keeps a wave on
+// fewer heads' rows, at the risk that a late group's heaviest units end
+// after everything else.  The host simulates that hand-out for both orders
+// (a unit costs its query steps plus a fixed kUnitFixedSteps) and groups
+// only when it costs at most 1 % more; the choice is cached per shape.
+constexpr int kUnitFixedSteps = 4;
+constexpr long long kMaxSimulatedUnits = 1 << 16;
+
+long long unit_makespan(int P, int nkb, int g, const std::vector<long long>& cost, int sms) {
+  std::priority_queue<long long, std::vector<long long>, std::greater<long long>> free_at;
+  for (int i = 0; i < sms; ++i) free_at.push(0);
+  long long end = 0;
+  for (int p0 = 0; p0 < P; p0 += g) {
+    const int gs = std::min(g, P - p0);
+    for (int kb = 0; kb < nkb; ++kb)
+      for (int j = 0; j < gs; ++j) {
+        const long long t = free_at.top() + cost[kb];
+        free_at.pop();
+        free_at.push(t);
+        end = std::max(end, t);
+      }
+  }
+  return end;
+}
+
+int choose_head_group(int P, int nkb, int n_qblk, int group, bool causal, int causal_off, int bm, int sms) {
+  if (P < 1 || nkb < 1 || sms < 1) return std::max(P, 1);
+  const int g = std::min(P, (sms + nkb - 1) / nkb);
+  if (g >= P || (long long)P * nkb > kMaxSimulatedUnits) return P;
+  struct Entry {
+    int key[8];
+    int g;
+  };
+  static std::mutex mu;
+  static Entry cache[16];
+  static int n_cached = 0, next_slot = 0;
+  const int key[8] = {P, nkb, n_qblk, group, (int)causal, causal ? causal_off : 0, bm, sms};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n_cached; ++i)
+      if (std::equal(key, key + 8, cache[i].key)) return cache[i].g;
+  }
+  std::vector<long long> cost(nkb);
+  for (int kb = 0; kb < nkb; ++kb) {
+    // the kernels' own count: query blocks from the first one with a visible key
+    const int qb_start = causal ? std::max(0, (kb * 128 - causal_off) / bm) : 0;
+    cost[kb] = (long long)group * std::max(0, n_qblk - qb_start) + kUnitFixedSteps;
+  }
+  const long long all_heads = unit_makespan(P, nkb, P, cost, sms);
+  const long long grouped = unit_makespan(P, nkb, g, cost, sms);
+  const int chosen = grouped * 100 <= all_heads * 101 ? g : P;
+  std::lock_guard<std::mutex> lk(mu);
+  Entry& e = cache[next_slot];
+  std::copy(key, key + 8, e.key);
+  e.g = chosen;
+  next_slot = (next_slot + 1) % 16;
+  n_cached = std::min(n_cached + 1, 16);
+  return chosen;
+}
+
 // Row length of the transposed dQ accumulator: a multiple of 32 queries, so
 // that its rows are 128-byte aligned for the TMA reduce-add.
 inline uint64_t dqt_row(int Nq) { return ((uint64_t)Nq + 31) & ~uint64_t(31); }
@@ -1201,6 +1291,7 @@ int launch(const void* q, const void* k, const void* v, const void* o, const voi
     a.scale_log2 = scale * kLog2e;
     const long long units = (long long)a.n_kblk * Hkv * B;
     if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    a.head_group = choose_head_group(Hkv * B, a.n_kblk, a.n_qblk, a.group, CAUSAL, a.causal_off, kBM, sms);
     if constexpr (kDqt) {
       using C = CfgT<CAUSAL>;
       static int attr_done = 0;

@@ -164,3 +164,26 @@ def test_long_context_gqa_workload_sampled():
     _grads_check(dq[:, r, 12:16], rq[:, :, 12:16], "dQ long-context sampled rows, heads 12-15")
     _grads_check(dk[:, kk, 3], rk[:, :, 3], "dK long-context sampled keys, KV head 3")
     _grads_check(dv[:, kk, 3], rv[:, :, 3], "dV long-context sampled keys, KV head 3")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_head_grouped_unit_order_sampled(D):
+    """Non-causal, B1, Hq = Hkv = 3, N = 9600: 75 key blocks per head, so the
+    unit order takes the heads two at a time (ceil(148 / 75) = 2, and with
+    equal units grouping costs nothing), which leaves a last group of one
+    head.  dQ of sampled query rows of every head, and dK, dV of sampled key
+    rows of the last group's head (2) and of the first group's second head (1),
+    against the oracle."""
+    N, H = 9600, 3
+    scale = 1.0 / math.sqrt(D)
+    q, k, v, do = inputs.bwd_inputs(1, H, H, N, N, D, seed=97)
+    dq, dk, dv = _run(q, k, v, do, False, scale)
+    rows = np.array([0, 1, 63, 64, 4800, N - 65, N - 1])
+    keys = np.array([0, 127, 128, 5000, 9471, 9472, N - 1])
+    for kvh in (2, 1):
+        rq, rk, rv = oracle.attention_bwd(to_np64(q), to_np64(k), to_np64(v), to_np64(do), False, scale,
+                                          q_rows=rows, k_rows=keys, kv_heads=[kvh])
+        r, kk = torch.as_tensor(rows), torch.as_tensor(keys)
+        _grads_check(dq.cpu()[:, r, kvh], rq[:, :, kvh], f"dQ sampled rows, head {kvh}, D={D}")
+        _grads_check(dk.cpu()[:, kk, kvh], rk[:, :, kvh], f"dK sampled keys, KV head {kvh}, D={D}")
+        _grads_check(dv.cpu()[:, kk, kvh], rv[:, :, kvh], f"dV sampled keys, KV head {kvh}, D={D}")
