@@ -139,9 +139,13 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // The kernels work on query units: with s_q query tokens per sequence, unit
-// u = b * s_q + i is query token i of sequence b.  The s_q tokens are the last
-// s_q cached tokens, so unit u sees positions 0 .. L_b - s_q + i (the causal
-// mask aligned to the bottom-right corner) of block-table row b.
+// u = i * n_seq + b is query token i of sequence b (token-major), and its
+// rows of q, o and lse are b * s_q + i.  The s_q tokens are the last s_q
+// cached tokens, so unit u sees positions 0 .. L_b - s_q + i (the causal mask
+// aligned to the bottom-right corner) of block-table row b.  Token-major
+// order puts the s_q units of a sequence 1/s_q of the split plan apart, so
+// CTA pairs that far apart walk the same pages at about the same time and
+// the later read of a page comes from L2.
 struct Args {
   const __nv_bfloat16* q;        // [B * s_q, Hq, DK]
   const uint8_t* kv;             // [num_pages, PAGE, DK] (only for L2 prefetches)
@@ -154,9 +158,14 @@ struct Args {
   float* ws_o;                   // [2 * pairs, Hq, DV]
   int* status;
   int B;                         // query units (sequences x s_q)
-  int s_q, max_pages, num_pages, pairs;
+  int s_q, n_seq, max_pages, num_pages, pairs;
   float scale_log2;
 };
+
+__device__ __forceinline__ int unit_seq(const Args& a, int u) { return u % a.n_seq; }
+__device__ __forceinline__ int unit_tok(const Args& a, int u) { return u / a.n_seq; }
+// Row of unit u in q [B, s_q, Hq, DK], o and lse.
+__device__ __forceinline__ int unit_row(const Args& a, int u) { return unit_seq(a, u) * a.s_q + unit_tok(a, u); }
 
 // Pages a sequence contributes (its length clamped to the block table).
 __device__ __forceinline__ int seq_pages(int L, int max_pages) {
@@ -174,7 +183,7 @@ __device__ __forceinline__ int seq_len_eff(int L, int max_pages) {
 // Positions unit u attends to: its sequence's length clamped to the block
 // table, minus the query tokens after it.
 __device__ __forceinline__ int unit_len(const Args& a, int u) {
-  const int L = seq_len_eff(a.seqlens[u / a.s_q], a.max_pages) - (a.s_q - 1 - u % a.s_q);
+  const int L = seq_len_eff(a.seqlens[unit_seq(a, u)], a.max_pages) - (a.s_q - 1 - unit_tok(a, u));
   return L > 0 ? L : 0;
 }
 
@@ -238,7 +247,7 @@ struct PageCursor {
     more = w.next(sb, g0, g1);
     if (more) {
       gp = g0;
-      row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages - pref[sb];
+      row = a.block_table + (size_t)unit_seq(a, sb) * a.max_pages - pref[sb];
     }
   }
   __device__ int next_with(const Args& a) {
@@ -249,7 +258,7 @@ struct PageCursor {
       more = w.next(sb, g0, g1);
       if (more) {
         gp = g0;
-        row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages - pref[sb];
+        row = a.block_table + (size_t)unit_seq(a, sb) * a.max_pages - pref[sb];
       }
     }
     return page;
@@ -301,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   {
     bool bad = false;
     for (int u = threadIdx.x; u < a.B; u += THREADS) {
-      const int L = a.seqlens[u / a.s_q];
+      const int L = a.seqlens[unit_seq(a, u)];
       pref[u + 1] = seq_pages(unit_len(a, u), a.max_pages);
       bad |= (L < 0) || ((long long)L > (long long)a.max_pages * PAGE);
     }
@@ -365,7 +374,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(bar(B_QE), (seg & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(bar(B_QF), Q_BYTES);
         for (int ch = 0; ch < Q_SMEM_CHUNKS; ++ch)
-          tma_load_2d(base + OFF_Q + ch * Q_CHUNK_BYTES, &tm_q, bar(B_QF), ch * 64, sb * HQ);
+          tma_load_2d(base + OFF_Q + ch * Q_CHUNK_BYTES, &tm_q, bar(B_QF), ch * 64, unit_row(a, sb) * HQ);
         q_last = seg;
         for (int gp = g0; gp < g1; ++gp, ++g) {
           int page = ids[0];
@@ -408,7 +417,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       int issued = 0;
       while (ok && w.next(sb, g0, g1)) {
-        const int32_t* row = a.block_table + (size_t)(sb / a.s_q) * a.max_pages;
+        const int32_t* row = a.block_table + (size_t)unit_seq(a, sb) * a.max_pages;
         for (int gp = g0; gp < g1; ++gp, ++g) {
           int page = row[gp - pref[sb]];
           if (page < 0 || page >= a.num_pages) page = 0;   // recorded by the rest producer
@@ -513,7 +522,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Q dims 320..575 of unit u's head into TMEM, half per group; the score
     // MMAs of segment s+1 wait for it (barrier QT).
     auto write_q_tmem = [&](int u) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)u * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)unit_row(a, u) * HQ + h) * DK + 64 * Q_SMEM_CHUNKS);
 #pragma unroll
       for (int cc = 0; cc < Q_TMEM_DIMS / 128; ++cc) {
         const int c = grp * (Q_TMEM_DIMS / 128) + cc;
@@ -650,6 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // of 32 rows x 16 bytes.
       const uint32_t xt = base + OFF_XPOSE + (uint32_t)((grp * 4 + q4) * XPOSE_BYTES);
       const int row0 = q4 * 32;   // first head of this warp
+      const int orow = unit_row(a, sb);
 #pragma unroll 1
       for (int c = 0; c < 128 / 32; ++c) {
         uint32_t o[32];
@@ -669,7 +679,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int r = 8 * j + (lane >> 2), u = lane & 3;
             uint32_t v0, v1, v2, v3;
             ld_shared_v4(xt + r * 128 + ((u ^ (r & 7)) * 16), v0, v1, v2, v3);
-            *reinterpret_cast<uint4*>(a.o + ((size_t)sb * HQ + row0 + r) * DV + col + 8 * u) = make_uint4(v0, v1, v2, v3);
+            *reinterpret_cast<uint4*>(a.o + ((size_t)orow * HQ + row0 + r) * DV + col + 8 * u) = make_uint4(v0, v1, v2, v3);
           }
         } else {
 #pragma unroll
@@ -692,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();   // the tile is rewritten by the next chunk
       }
       if (half == 0 && grp == 0) {
-        if (full) a.lse[(size_t)sb * HQ + h] = lse;
+        if (full) a.lse[(size_t)orow * HQ + h] = lse;
         else a.ws_lse[(size_t)slot * HQ + h] = lse;
       }
       tc_fence_before();
@@ -744,15 +754,16 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
   // Launched as a programmatic dependent of the split kernel: wait here until
   // that grid has completed and its writes are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int b = blockIdx.x;
+  const int b = blockIdx.x;                 // query unit
+  const int orow = unit_row(a, b);          // its row of o and lse
   const int h0 = blockIdx.y * COMBINE_HEADS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = a.ws_pref[a.B];
   const int s0 = a.ws_pref[b], s1 = a.ws_pref[b + 1];
   if (s1 == s0) {
     for (int i = tid; i < COMBINE_HEADS * DV; i += COMBINE_THREADS)
-      a.o[((size_t)b * HQ + h0) * DV + i] = __float2bfloat16(0.f);
-    if (tid < COMBINE_HEADS) a.lse[(size_t)b * HQ + h0 + tid] = -INFINITY;
+      a.o[((size_t)orow * HQ + h0) * DV + i] = __float2bfloat16(0.f);
+    if (tid < COMBINE_HEADS) a.lse[(size_t)orow * HQ + h0 + tid] = -INFINITY;
     return;
   }
   const int p_lo = pair_of_page(s0, T, a.pairs), p_hi = pair_of_page(s1 - 1, T, a.pairs);
@@ -803,7 +814,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
     for (int j = lane; j < nparts; j += 32) w_s[hh][j] *= inv;
-    if (lane == 0) a.lse[(size_t)b * HQ + h0 + hh] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    if (lane == 0) a.lse[(size_t)orow * HQ + h0 + hh] = sum > 0.f ? mx + logf(sum) : -INFINITY;
   }
   __syncthreads();
   // COMBINE_HEADS x 512 columns as float4 groups: thread tid owns groups
@@ -847,7 +858,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
 #pragma unroll
   for (int k = 0; k < OUT_PER_THREAD; ++k) {
     const int g = tid + COMBINE_THREADS * k;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)b * HQ + h0 + hh_of[k]) * DV + (g % (DV / 4)) * 4);
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)orow * HQ + h0 + hh_of[k]) * DV + (g % (DV / 4)) * 4);
     dst[0] = __floats2bfloat162_rn(acc[k].x, acc[k].y);
     dst[1] = __floats2bfloat162_rn(acc[k].z, acc[k].w);
   }
@@ -944,6 +955,7 @@ extern "C" int attn_decode_paged_mtp(const void* q, const void* kv_pages, const 
   a.status = status;
   a.B = units;
   a.s_q = s_q;
+  a.n_seq = B;
   a.max_pages = max_pages_per_seq;
   a.num_pages = num_pages;
   a.pairs = pairs;
