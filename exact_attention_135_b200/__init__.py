@@ -19,9 +19,9 @@ import re
 
 import torch
 
-__all__ = ["fwd", "decode_paged", "decode_paged_mtp", "decode_paged_noalloc", "decode_workspace_size",
-           "decode_mtp_workspace_size", "decode_paged_gqa", "decode_gqa_workspace_size", "read_device_status",
-           "library", "AttnError", "exported_symbols", "STATUS"]
+__all__ = ["fwd", "fwd_fp8", "bwd", "bwd_workspace_size", "bwd_head_group", "decode_paged", "decode_paged_mtp",
+           "decode_paged_noalloc", "decode_workspace_size", "decode_mtp_workspace_size", "decode_paged_gqa",
+           "decode_gqa_workspace_size", "read_device_status", "library", "AttnError", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libattn_b200.so")
@@ -60,6 +60,7 @@ _SIGNATURES = {
     "attn_decode_paged_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _f, _f, _f, _vp, _vp] + [_i] * 7 + [_f, _vp]),
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "attn_bwd_head_group": (_i, [_i] * 8),
     "attn_bwd": (_i, [_vp] * 9 + [_i] * 8 + [_f, _vp, _sz, _vp]),
 }
 
@@ -179,6 +180,12 @@ def fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float,
 
 def bwd_workspace_size(B: int, Hq: int, Nq: int, D: int) -> int:
     return int(library().attn_bwd_workspace_size(B, Hq, Nq, D))
+
+
+def bwd_head_group(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, D: int, causal: bool, sm_count: int) -> int:
+    """(batch, KV head) pairs per group in bwd's unit order for this shape
+    on a device with sm_count SMs (host-only; 0 for rejected arguments)."""
+    return int(library().attn_bwd_head_group(B, Hq, Hkv, Nq, Nk, D, int(bool(causal)), sm_count))
 
 
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,

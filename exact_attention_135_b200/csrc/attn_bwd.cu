@@ -1333,6 +1333,17 @@ extern "C" size_t attn_bwd_workspace_size(int B, int Hq, int Nq, int D) {
   return ea::bwd::workspace_bytes(B, Hq, Nq, D);
 }
 
+extern "C" int attn_bwd_head_group(int B, int Hq, int Hkv, int Nq, int Nk, int D, int causal, int sm_count) {
+  using namespace ea::bwd;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 1 || Hq % Hkv != 0 || sm_count < 1) return 0;
+  if (D != 64 && D != 128) return 0;
+  if ((long long)B * Hkv > 0x7fffffffLL) return 0;
+  // the query block of the kernel that attn_bwd runs for D
+  const int bm = D == 128 ? CfgT<true>::BM : Cfg<64, true>::BM;
+  return choose_head_group(B * Hkv, (Nk + 127) / 128, (Nq + bm - 1) / bm, Hq / Hkv, causal != 0, Nk - Nq, bm,
+                           sm_count);
+}
+
 extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                         const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
                         int D, int Dv, int causal, float scale, void* workspace, size_t workspace_bytes,

@@ -150,6 +150,21 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd_head_group: the unit order attn_bwd takes for this shape on a
+ * device with sm_count SMs.  Host-only: it launches nothing and needs no GPU.
+ * attn_bwd runs one CTA per (key block of 128 keys, KV head, batch) and hands
+ * the CTAs out g (batch, KV head) pairs at a time, key block slowest inside
+ * a group, so the causal blocks that see the most queries start first.
+ * Returns g: B * Hkv is key block slowest over every pair.  A smaller g,
+ * ceil(sm_count / key blocks), keeps fewer heads' Q, dO and dQ rows live in
+ * L2 at once.  It is taken only when a model of the block scheduler gives it
+ * at most 1 % more makespan.  In that model each unit goes, in order, to the
+ * SM that frees first and costs its query steps plus 4.  Returns 0 for
+ * arguments that attn_bwd would reject, and for Nk == 0 (no units).
+ */
+int attn_bwd_head_group(int B, int Hq, int Hkv, int Nq, int Nk, int D, int causal, int sm_count);
+
+/*
  * attn_decode_paged_workspace_size: bytes of device workspace that
  * attn_decode_paged needs for a batch of B sequences with Hq heads of width
  * Dv when it runs on CUDA device `device` (the split-KV plan depends on the
