@@ -64,7 +64,9 @@ NCU_TRAFFIC_BYTES = {
     "prefill": 364641536 + 105544448,   # attn_fwd_kernel<D=128, causal> (persistent), GQA N=16384 workload
     "prefill_c4": 151093504 + 101837824,   # attn_fwd_kernel<D=256> (persistent), MQA D=256 workload
     "prefill_c2": 37816320 + 63232,     # attn_fwd_kernel<D=64, causal> (persistent), GPT-2-small shape
-    "decode": 349552640 + 15395840,     # decode_split_kernel, MLA decode workload
+    # decode_split_kernel, MLA decode workload (with one token per sequence the
+    # token-major unit numbering is the identity, so its loads are unchanged)
+    "decode": 349552640 + 15395840,
     "mtp": 363760000 + 26660000,        # decode_split_kernel, MLA decode workload with 2 query tokens per sequence
     "gqa": 1357133568 + 4723712,        # gqa_decode_kernel, GQA-path decode workload
     "bwd": 665277184 + 338907392,       # attn_bwd_dqt_kernel<causal>, GQA N=16384 workload (backward)
