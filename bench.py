@@ -461,8 +461,14 @@ def run_gpu(args):
                           "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peaks_kind} HBM copy",
                           "traffic": traffic, "kernel": kernel},
              "e2e": e2e_obj(p, p.kv_bytes, "GB/s", 1e9)}
+        # against the nominal ~8 TB/s of HBM3e as well as the measured copy
+        o["roofline"]["frac_of_nominal_8tbs"] = round(gbs / 8000.0, 4)
         if hasattr(p, "flops"):
             o["roofline"]["tflops"] = round(p.flops / sec / 1e12, 1)
+            # combined roofline: the slower of moving the KV bytes at the HBM
+            # peak and doing the FLOPs at this line's bf16 peak, over the time
+            t_min = max(p.kv_bytes / (peaks["hbm_gbs"] * 1e9), p.flops / (bf16_peak * 1e12))
+            o["roofline"]["frac_of_combined"] = round(t_min / sec, 4)
         if extra:
             o.update(extra)
         return o
